@@ -1,0 +1,444 @@
+"""Benchmark of the B200 ConvTranspose library: one JSON line on rank 0.
+
+A step is one ``ct_run`` of the headline workload (2-D decoder upsample,
+fp16, X[8,256,64,64] * W[256,128,4,4], stride 2, pads 1 -> Y[8,128,128,128])
+with X resident in HBM: plan, output-size resolution and the weight pre-pack
+happen once, before timing, as they do for a deployed layer.  The metric is
+effective TFLOP/s = 2*N*C*(M/group)*prod(in)*prod(k) / time, summed over
+ranks.  Steps are CUDA-graph launches of one ct_run each, rotating over
+enough X/Y buffer sets that consecutive steps do not hit L2 (more bytes than
+the L2 holds between reuses).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun each rank runs its own replica of the workload (weak scaling:
+the batch is independent per GPU, no collective on the data path); the
+reported time is the max over ranks.  ``--impl reference`` times the fp64
+CPU oracle on a bounded sample of the same workload instead.
+"""
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from transposed_convolution_02_b200 import ct  # noqa: E402
+from transposed_convolution_02_b200.workloads import WORKLOADS, make_inputs  # noqa: E402
+
+HEADLINE = 2
+METRIC = "ConvTranspose effective TFLOP/s per config at 1 B200; % of tensor/HBM roofline"
+
+
+# ---------------------------------------------------------------------------
+# workload arithmetic used for reporting
+
+def workload_numbers(wl):
+    """Effective FLOP per pass and algorithmic bytes (X + W + bias + Y once)."""
+    n, c = wl.x_shape[0], wl.x_shape[1]
+    mg = wl.w_shape[1]
+    flop = 2 * n * c * mg * math.prod(wl.x_shape[2:]) * math.prod(wl.w_shape[2:])
+    eb = torch.finfo(wl.dtype).bits // 8
+    m = mg * wl.group
+    nbytes = eb * (math.prod(wl.x_shape) + math.prod(wl.w_shape) + (m if wl.bias else 0)
+                   + math.prod(wl.y_shape))
+    return flop, nbytes
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return dict(hbm_gbs=pk["hbm_gbs"], tc_tflops=pk["bf16_tflops"],
+                    tc_tflops_sustained=pk.get("bf16_tflops_sustained"),
+                    sm_max_mhz=pk.get("sm_max_mhz", 1965.0), source="measured")
+    return dict(hbm_gbs=6650.0, tc_tflops=1590.0, tc_tflops_sustained=1400.0,
+                sm_max_mhz=1965.0, source="fallback")
+
+
+def roofline_for(wl, seconds_per_launch, peaks, sms):
+    """Bound and achieved rate of the workload's dominant kernel."""
+    flop, nbytes = workload_numbers(wl)
+    if wl.dtype == torch.float32:
+        # FP32 FFMA peak: SMs x 128 lanes x 2 flop x max SM clock
+        peak = sms * 128 * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12
+        return dict(bound="alu", achieved=flop / seconds_per_launch / 1e12, peak=peak,
+                    unit="TFLOP/s", frac=(flop / seconds_per_launch / 1e12) / peak)
+    t_tc = flop / (peaks["tc_tflops"] * 1e12)
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    if t_tc >= t_hbm:
+        a = flop / seconds_per_launch / 1e12
+        return dict(bound="tensor", achieved=a, peak=peaks["tc_tflops"], unit="TFLOP/s",
+                    frac=a / peaks["tc_tflops"])
+    a = nbytes / seconds_per_launch / 1e9
+    return dict(bound="hbm", achieved=a, peak=peaks["hbm_gbs"], unit="GB/s",
+                frac=a / peaks["hbm_gbs"])
+
+
+def traffic_for(kernel):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel source
+    is unchanged since the capture (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f).get(kernel)
+    if not rec:
+        return None
+    src = os.path.join(ROOT, "transposed_convolution_02_b200", "csrc", rec["source"])
+    if not os.path.exists(src):
+        return None
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return rec["bytes_per_launch"] if h == rec["sha256_16"] else None
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML reads only; nothing is changed)
+
+class ClockSampler:
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, device_index):
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._h = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            idx = device_index
+            if vis:
+                ids = [v for v in vis.split(",") if v.strip()]
+                if device_index < len(ids) and ids[device_index].strip().isdigit():
+                    idx = int(ids[device_index])
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._h = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self._h is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._h is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+
+def build_op(wl, device):
+    x, w, b = make_inputs(wl)
+    op = ct.ConvTranspose(w.to(device), list(x.shape), b.to(device) if b is not None else None,
+                          strides=wl.strides, dilations=wl.dilations, pads=wl.pads,
+                          output_padding=wl.output_padding, auto_pad=wl.auto_pad,
+                          group=wl.group)
+    return op, x
+
+
+def time_device(wl, device, steps, warmup, l2_bytes, dist_max=None, sampler=None):
+    """Device time of `steps` ct_runs (CUDA graphs, rotating buffer sets)."""
+    op, x_cpu = build_op(wl, device)
+    xb = x_cpu.numel() * x_cpu.element_size()
+    yb = math.prod(op.y_shape) * x_cpu.element_size()
+    nsets = max(2, min(8, math.ceil(2 * l2_bytes / (xb + yb)) + 1))
+    free, _ = torch.cuda.mem_get_info(device)
+    while nsets > 1 and nsets * (xb + yb) > 0.6 * free:
+        nsets -= 1
+    xs = [x_cpu.to(device) for _ in range(nsets)]
+    ys = [torch.empty(op.y_shape, dtype=wl.dtype, device=device) for _ in range(nsets)]
+    graphs = []
+    s = torch.cuda.Stream(device)
+    s.wait_stream(torch.cuda.current_stream(device))
+    with torch.cuda.stream(s):
+        for i in range(nsets):       # warm the launch path before capture
+            op(xs[i], out=ys[i])
+    torch.cuda.current_stream(device).wait_stream(s)
+    torch.cuda.synchronize(device)
+    for i in range(nsets):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            op(xs[i], out=ys[i])
+        graphs.append(g)
+    for j in range(warmup):
+        graphs[j % nsets].replay()
+    if dist_max is not None:
+        dist_max("barrier")
+    torch.cuda.synchronize(device)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    ctx = sampler if sampler is not None else _Null()
+    with ctx:
+        start.record()
+        for j in range(steps):
+            graphs[(warmup + j) % nsets].replay()
+        end.record()
+        torch.cuda.synchronize(device)
+    if dist_max is not None:
+        dist_max("barrier")
+    ms = start.elapsed_time(end)
+    info = dict(kernel=op.kernel, launches_per_step=op.launches, sets=nsets,
+                set_bytes=xb + yb)
+    del graphs
+    return ms, info
+
+
+class _Null:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        return False
+
+
+def time_e2e(wl, device, steps, warmup):
+    """Through the public API with host buffers: pinned X -> device, ct_run,
+    Y -> pinned host, all inside the timed region every step."""
+    op, x_cpu = build_op(wl, device)
+    xh = x_cpu.pin_memory()
+    yh = torch.empty(op.y_shape, dtype=wl.dtype).pin_memory()
+    xd = torch.empty_like(x_cpu, device=device)
+    yd = torch.empty(op.y_shape, dtype=wl.dtype, device=device)
+
+    def step():
+        xd.copy_(xh, non_blocking=True)
+        op(xd, out=yd)
+        yh.copy_(yd, non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(device)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(steps):
+        step()
+    end.record()
+    torch.cuda.synchronize(device)
+    return start.elapsed_time(end), xh.numel() * xh.element_size(), yh.numel() * yh.element_size()
+
+
+# ---------------------------------------------------------------------------
+# the oracle on the host cores (reported baseline / reference arm)
+
+def oracle_sample(wl, target_s=12.0):
+    """Time the fp64 oracle on a bounded sample of the workload.
+
+    The sample is batch image 0, the first m' output channels of every group
+    (m' = as many as there are cores, at most M/group: the oracle's threads
+    split the work by output plane) and the first h' positions of the first
+    spatial axis of X, h' sized from a one-row calibration run so the sample
+    takes about ``target_s``.  Returns (TFLOP/s, cores, description, seconds).
+    """
+    from oracle import Attrs, conv_transpose_ref
+    x, w, b = make_inputs(wl)
+    x = x[:1].double().numpy()
+    w = w.double().numpy()
+    b = b.double().numpy() if b is not None else None
+    g = wl.group
+    mg_full = wl.w_shape[1]
+    cores = len(os.sched_getaffinity(0))
+    os.environ.setdefault("OMP_NUM_THREADS", str(cores))
+    mg = max(1, min(mg_full, math.ceil(cores / g)))
+    ws = np.ascontiguousarray(w[:, :mg])
+    bs = None
+    if b is not None:
+        bs = np.ascontiguousarray(b.reshape(g, mg_full)[:, :mg].reshape(-1))
+    attrs = Attrs(strides=wl.strides, dilations=wl.dilations, pads=wl.pads,
+                  output_padding=wl.output_padding, auto_pad=wl.auto_pad, group=g)
+    rows = x.shape[2]
+
+    def run(h):
+        xs = np.ascontiguousarray(x[:, :, :h])
+        t0 = time.perf_counter()
+        conv_transpose_ref(xs, ws, bs, attrs)
+        dt = time.perf_counter() - t0
+        flop = 2 * xs.shape[1] * mg * math.prod(xs.shape[2:]) * math.prod(w.shape[2:])
+        return dt, flop
+
+    dt, flop = run(1)
+    h = int(max(1, min(rows, round(target_s / max(dt, 1e-4)))))
+    if h > 1:
+        dt, flop = run(h)
+    desc = ("batch image 0 of %d, %d of %d output channels per group, first %d of %d "
+            "positions on the first spatial axis (%.3f GFLOP), %d OpenMP threads"
+            % (wl.x_shape[0], mg, mg_full, h, rows, flop / 1e9, cores))
+    return flop / dt / 1e12, cores, desc, dt
+
+
+# ---------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", type=int, default=HEADLINE)
+    ap.add_argument("--no-others", action="store_true",
+                    help="skip the secondary per-workload measurements")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    wl = WORKLOADS[args.workload]
+    flop, nbytes = workload_numbers(wl)
+    config = {"workload": wl.name, "x": list(wl.x_shape), "w": list(wl.w_shape),
+              "y": list(wl.y_shape), "global_batch": wl.x_shape[0] * max(world, 1),
+              "parallelism": "dp%d (independent replica per GPU)" % max(world, 1)}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        per_step = []
+        info = None
+        budget = min(12.0, 150.0 / (args.steps + args.warmup))
+        for _ in range(args.warmup):
+            oracle_sample(wl, target_s=budget)
+        for _ in range(args.steps):
+            v, cores, desc, dt = oracle_sample(wl, target_s=budget)
+            per_step.append((v, dt))
+            info = (cores, desc)
+        v = statistics.median([p[0] for p in per_step])
+        line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s",
+                "n_gpus": 0, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": 1e3 * statistics.median([p[1] for p in per_step]),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "f64", "data": "synthetic (seeded, workload distributions)",
+                "config": config,
+                "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": info[0],
+                                 "kind": "oracle", "sample": info[1]},
+                "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    dist_max = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+        def dist_max(what, value=None):
+            if what == "barrier":
+                dist.barrier()
+                return None
+            t = torch.tensor([value], dtype=torch.float64, device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            return float(t.item())
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    props = torch.cuda.get_device_properties(device)
+    l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20)
+    peaks = load_peaks()
+
+    sampler = ClockSampler(local)
+    ms, info = time_device(wl, device, args.steps, args.warmup, l2, dist_max, sampler)
+    if dist_max is not None:
+        ms = dist_max("max", ms)
+    sec_per_step = ms / 1e3 / args.steps
+    value = flop * max(world, 1) / sec_per_step / 1e12
+    roof = roofline_for(wl, sec_per_step, peaks, props.multi_processor_count)
+    roof["peak_source"] = peaks["source"] + " (burst)"
+    roof["traffic"] = traffic_for(info["kernel"])
+    roof["kernel"] = info["kernel"]
+    roof["per_launch_us"] = sec_per_step * 1e6 / max(1, info["launches_per_step"])
+
+    e2e_steps = max(3, min(args.steps, 50))
+    ems, hb, db = time_e2e(wl, device, e2e_steps, 3)
+    if dist_max is not None:
+        ems = dist_max("max", ems)
+    e2e_value = flop * max(world, 1) / (ems / 1e3 / e2e_steps) / 1e12
+
+    others = {}
+    if not args.no_others:
+        for wid in sorted(WORKLOADS):
+            if wid == args.workload:
+                continue
+            owl = WORKLOADS[wid]
+            ofl, _ = workload_numbers(owl)
+            osteps = 20 if owl.dtype == torch.float32 and wid == 4 else 200
+            oms, oinfo = time_device(owl, device, osteps, 5, l2, dist_max)
+            if dist_max is not None:
+                oms = dist_max("max", oms)
+            osec = oms / 1e3 / osteps
+            oroof = roofline_for(owl, osec, peaks, props.multi_processor_count)
+            others[str(wid)] = {"workload": owl.name, "kernel": oinfo["kernel"],
+                                "us_per_step": osec * 1e6, "tflops": ofl / osec / 1e12,
+                                "roofline": oroof}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, cores, desc, dt = oracle_sample(wl)
+        cpu = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc}
+
+    if rank == 0:
+        clocks = sampler.summary()
+        line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": max(world, 1),
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "f16" if wl.dtype == torch.float16 else "f32",
+                "data": "synthetic (seeded; X~N(0,1), W~N(0,1/32), bias~N(0,0.1))",
+                "config": dict(config, l2="rotating %d X/Y buffer sets of %.1f MB (> L2 %d MB "
+                               "between reuses)" % (info["sets"], info["set_bytes"] / 1e6,
+                                                    l2 // 2 ** 20),
+                               kernel=info["kernel"], launch="CUDA graph per step"),
+                "roofline": roof,
+                "cpu_baseline": cpu,
+                "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": hb,
+                        "d2h_bytes_per_step": db},
+                "gpu_launches": args.steps * info["launches_per_step"],
+                "clocks": clocks,
+                "others": others}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

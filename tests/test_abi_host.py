@@ -1,0 +1,184 @@
+"""Host-side checks of libct.so that need no GPU: the library loads, exports
+every entry point include/ct.h declares, and its resolver agrees with the
+oracle's independent resolver on random attribute sets."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+from cases import attrs_of, random_case
+from oracle import Attrs, ResolveError, resolve_full
+from transposed_convolution_02_b200 import ct
+from transposed_convolution_02_b200.workloads import WORKLOADS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            names |= set(re.findall(r"CT_API\s+[\w\s\*]*?\b(ct_\w+)\s*\(", src))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    L = ct.lib()
+    declared = _declared_symbols()
+    assert declared, "no declarations found"
+    for name in declared:
+        assert hasattr(L, name), name
+    assert declared == set(ct.EXPORTED)
+
+
+def test_status_strings():
+    for code in range(0, 11):
+        assert ct.ct_status_string(code)
+    assert ct.ct_status_string(0) == "ok"
+
+
+def _desc_from_case(case, layout="nchw", dtype=torch.float32):
+    x_shape, w_shape = list(case["x_shape"]), list(case["w_shape"])
+    if layout == "nhwc":
+        x_shape = [x_shape[0]] + x_shape[2:] + [x_shape[1]]
+        w_shape = [w_shape[0]] + w_shape[2:] + [w_shape[1]]
+    m = case["w_shape"][1] * case["group"]
+    return ct.make_desc(x_shape, w_shape, dtype=dtype, layout=layout,
+                        strides=case["strides"], dilations=case.get("dilations"),
+                        pads=case.get("pads"), output_padding=case.get("output_padding"),
+                        auto_pad=case.get("auto_pad", "NOTSET"), group=case["group"],
+                        bias_len=m if case.get("bias") else 0,
+                        kernel_shape=case.get("kernel_shape"),
+                        output_shape=case.get("output_shape"))
+
+
+@pytest.mark.parametrize("layout", ["nchw", "nhwc"])
+def test_resolver_agrees_with_oracle(layout):
+    rng = np.random.default_rng(99)
+    modes = ["NOTSET", "NOTSET", "SAME_UPPER", "SAME_LOWER", "VALID"]
+    n_ok = n_err = 0
+    for _ in range(3000):
+        case = random_case(rng, pads=(-2, 4))
+        r = len(case["strides"])
+        case["auto_pad"] = str(rng.choice(modes))
+        if case["auto_pad"] != "NOTSET" and rng.random() < 0.8:
+            case["pads"] = [0] * (2 * r)
+        # perturb to reach the error paths too
+        u = rng.random()
+        if u < 0.05:
+            case["output_padding"][0] = max(case["strides"][0], case["dilations"][0])
+        elif u < 0.10:
+            case["kernel_shape"] = [k + 1 for k in case["w_shape"][2:]]
+        elif u < 0.25:
+            case["output_shape"] = [int(v) for v in rng.integers(1, 30, size=r)]
+        elif u < 0.28:
+            case["strides"][0] = 0
+        try:
+            yshape, res = resolve_full(case["x_shape"], case["w_shape"], attrs_of(case))
+            want = ("ok", yshape, res.pad_begin, res.pad_end)
+        except ResolveError:
+            want = ("err",)
+        d = _desc_from_case(case, layout)
+        try:
+            ys, pb, pe = ct.ct_output_shape(d)
+            if layout == "nhwc":
+                ys = [ys[0], ys[-1]] + ys[1:-1]
+            got = ("ok", ys, pb, pe)
+        except ct.CtError:
+            got = ("err",)
+        assert got == want, (case, got, want)
+        n_ok += want[0] == "ok"
+        n_err += want[0] == "err"
+    assert n_ok > 1000 and n_err > 100
+
+
+def test_error_classes():
+    base = dict(x_shape=[1, 4, 5], w_shape=[4, 3, 3], strides=[2], pads=[1, 1], group=2)
+
+    def status(**over):
+        c = dict(base)
+        c.update(over)
+        d = _desc_from_case(c)
+        for k in ("bias_len",):
+            if k in over:
+                setattr(d, k, over[k])
+        try:
+            ct.ct_output_shape(d)
+            return 0
+        except ct.CtError as e:
+            return e.status
+
+    assert status() == 0
+    assert status(group=3) == 1                       # C % group
+    assert status(w_shape=[3, 3, 3]) == 1             # W[0] != C
+    assert status(bias_len=5) == 1                    # bias length != M = 6
+    assert status(output_padding=[2]) == 4            # op >= max(s, d)
+    assert status(strides=[0]) == 4
+    assert status(kernel_shape=[2]) == 4
+    assert status(auto_pad="SAME_UPPER") == 4         # pads with auto_pad
+    d = _desc_from_case(base)
+    d.rank = 4
+    with pytest.raises(ct.CtError) as e:
+        ct.ct_output_shape(d)
+    assert e.value.status == 2
+    d = _desc_from_case(base)
+    d.dtype = 7
+    with pytest.raises(ct.CtError) as e:
+        ct.ct_output_shape(d)
+    assert e.value.status == 3
+
+
+@pytest.mark.parametrize("wid", sorted(WORKLOADS))
+def test_workload_shapes_and_plan(wid):
+    wl = WORKLOADS[wid]
+    case = dict(x_shape=wl.x_shape, w_shape=wl.w_shape, strides=wl.strides,
+                dilations=wl.dilations, pads=wl.pads, output_padding=wl.output_padding,
+                auto_pad=wl.auto_pad, group=wl.group, bias=wl.bias)
+    d = _desc_from_case(case, dtype=wl.dtype)
+    ys, pb, pe = ct.ct_output_shape(d)
+    assert ys == list(wl.y_shape)
+    plan = ct.ct_plan(d)
+    try:
+        assert ct.ct_plan_kernel(plan) in ("generic", "dense_tc", "fp32_gemm", "grouped")
+        assert ct.ct_prepacked_weight_bytes(plan) > 0
+        assert ct.ct_workspace_bytes(plan) >= 0
+    finally:
+        ct.ct_plan_destroy(plan)
+
+
+def test_forced_generic_and_unsupported():
+    case = dict(x_shape=[1, 4, 5], w_shape=[4, 3, 3], strides=[2], pads=[1, 1], group=2)
+    d = _desc_from_case(case)
+    d.algo = ct.ALGO["generic"]
+    plan = ct.ct_plan(d)
+    assert ct.ct_plan_kernel(plan) == "generic"
+    ct.ct_plan_destroy(plan)
+    d.algo = ct.ALGO["dense_tc"]    # fp32 grouped: the tensor-core kernel cannot serve it
+    with pytest.raises(ct.CtError) as e:
+        ct.ct_plan(d)
+    assert e.value.status == 9
+
+
+def test_run_argument_checks_without_device():
+    case = dict(x_shape=[1, 4, 5], w_shape=[4, 3, 3], strides=[2], pads=[1, 1], group=2,
+                bias=True)
+    plan = ct.ct_plan(_desc_from_case(case))
+    try:
+        P = ctypes.c_void_p
+        # NULL y, NULL bias while a bias is declared: rejected before any device call
+        with pytest.raises(ct.CtError) as e:
+            ct.ct_run(plan, P(4096), P(4096), P(4096), P(0), P(0), P(0))
+        assert e.value.status == 6
+        with pytest.raises(ct.CtError) as e:
+            ct.ct_run(plan, P(4096), P(4096), P(0), P(4096), P(0), P(0))
+        assert e.value.status == 6
+        with pytest.raises(ct.CtError) as e:   # fp32 y at an odd address
+            ct.ct_run(plan, P(4096), P(4096), P(4096), P(4097), P(0), P(0))
+        assert e.value.status == 5
+    finally:
+        ct.ct_plan_destroy(plan)
