@@ -317,6 +317,8 @@ def main():
     ap.add_argument("--no-others", action="store_true",
                     help="skip the secondary per-workload measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--plain", action="store_true",
+                    help="profiling mode: eager ct_run launches of one workload, nothing else")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -354,6 +356,19 @@ def main():
                 "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
+        return
+
+    if args.plain:
+        device = torch.device("cuda", local)
+        torch.cuda.set_device(device)
+        op, x_cpu = build_op(wl, device)
+        x = x_cpu.to(device)
+        y = torch.empty(op.y_shape, dtype=wl.dtype, device=device)
+        for _ in range(args.warmup + args.steps):
+            op(x, out=y)
+        torch.cuda.synchronize(device)
+        print(json.dumps({"plain": wl.name, "kernel": op.kernel, "launches": op.launches,
+                          "runs": args.warmup + args.steps}), flush=True)
         return
 
     dist_max = None

@@ -84,7 +84,9 @@ typedef enum ct_algo {
     CT_ALGO_GENERIC = 1,   /* per-output gather, any shape */
     CT_ALGO_DENSE_TC = 2,  /* fp16 group-1 phase GEMM on tcgen05 tensor cores */
     CT_ALGO_FP32_GEMM = 3, /* fp32 group-1 register-tiled FFMA phase GEMM */
-    CT_ALGO_GROUPED = 4    /* fp16 grouped phase kernel (mma.sync), small per-group slabs */
+    CT_ALGO_GROUPED = 4,   /* fp16 grouped phase kernel (mma.sync), small per-group slabs */
+    CT_ALGO_DENSE_TC_PERTAP = 5 /* fp16 group-1 tcgen05 phase GEMM, one input load per tap
+                                   (the general fallback of CT_ALGO_DENSE_TC) */
 } ct_algo;
 
 /* One ConvTranspose call.  Every array has 3 slots; only the first `rank`

@@ -81,7 +81,7 @@ def full_parity(case, dtype, seed, layout="nchw", algo="auto", expect_kernel=Non
     if layout == "nhwc":
         ref = np.moveaxis(ref, 1, -1)
         absacc = np.moveaxis(absacc, 1, -1)
-    return op, check_close(y, ref, absacc, dtype, str(case))
+    return op, check_close(y, ref, absacc, dtype, "%s %s %s" % (case, layout, op.kernel))
 
 
 def sampled_points(y_shape_cf, rng, n_random=1500):

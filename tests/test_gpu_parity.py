@@ -100,3 +100,60 @@ def test_workload_full_size(wid):
         bb = b.cuda().view(1, -1, 1, 1).expand(y.shape[0], -1, y.shape[2], y.shape[3])
         assert torch.equal(y[:, :, 0::2, :], bb[:, :, 0::2, :])
         assert torch.equal(y[:, :, :, 0::2], bb[:, :, :, 0::2])
+
+
+def _dense_case(rng, lim_in):
+    case = random_case(rng, groups=(1,), max_cg=1, max_mg=1, lim_in=lim_in,
+                       lim_k={1: 9, 2: 5, 3: 3})
+    c = int(rng.choice([8, 16, 24, 64, 72, 136]))
+    m = int(rng.choice([1, 7, 16, 33, 64, 100, 128, 200]))
+    case["x_shape"][1] = c
+    case["w_shape"][0] = c
+    case["w_shape"][1] = m
+    return case
+
+
+@pytest.mark.parametrize("layout", ["nchw", "nhwc"])
+def test_dense_tc_random_sweep(layout):
+    """fp16 group-1 shapes on the tcgen05 halo phase-GEMM kernel (falling back
+    to the per-tap kernel for rows narrower than 8 J positions): ranks 1-3,
+    strides/dilations up to 3-4, negative and asymmetric pads, M not a
+    multiple of 16, C spanning partial 64-channel blocks, phases without
+    taps (filled with the bias)."""
+    rng = np.random.default_rng(300 + (layout == "nhwc"))
+    kernels = []
+    for i in range(40):
+        case = _dense_case(rng, {1: 400, 2: 40, 3: 12})
+        op, _ = full_parity(case, torch.float16, 7000 + i, layout, algo="dense_tc")
+        assert op.kernel in ("dense_tc", "dense_tc_pertap")
+        kernels.append(op.kernel)
+    assert kernels.count("dense_tc") >= 20, kernels
+
+
+@pytest.mark.parametrize("layout", ["nchw", "nhwc"])
+def test_dense_tc_pertap_random_sweep(layout):
+    """The general per-tap tcgen05 kernel on the same kind of shapes."""
+    rng = np.random.default_rng(400 + (layout == "nhwc"))
+    for i in range(30):
+        case = _dense_case(rng, {1: 300, 2: 20, 3: 7})
+        full_parity(case, torch.float16, 8000 + i, layout, algo="dense_tc_pertap",
+                    expect_kernel="dense_tc_pertap")
+
+
+def test_dense_tc_dead_phases_and_degenerate():
+    # stride 2, dilation 2: taps land only on odd outputs; the rest is bias
+    case = dict(x_shape=[2, 32, 9, 10], w_shape=[32, 24, 3, 3], strides=[2, 2],
+                dilations=[2, 2], auto_pad="SAME_UPPER", bias=True)
+    for algo in ("dense_tc", "dense_tc_pertap"):
+        full_parity(case, torch.float16, 41, "nchw", algo=algo, expect_kernel=algo)
+    # 1x1 kernel, stride 1 (the plain GEMM case), and a rank-1 long signal
+    for algo in ("dense_tc", "dense_tc_pertap"):
+        full_parity(dict(x_shape=[3, 64, 17, 9], w_shape=[64, 48, 1, 1], strides=[1, 1],
+                         bias=True), torch.float16, 42, "nchw", algo=algo, expect_kernel=algo)
+        full_parity(dict(x_shape=[2, 16, 1000], w_shape=[16, 8, 16], strides=[8], pads=[4, 4],
+                         bias=True), torch.float16, 43, "nhwc", algo=algo, expect_kernel=algo)
+    # many M-tiles in y with a ragged tail, several channel blocks, both layouts
+    for layout in ("nchw", "nhwc"):
+        full_parity(dict(x_shape=[2, 136, 23, 70], w_shape=[136, 96, 4, 4], strides=[2, 2],
+                         pads=[1, 1, 1, 1], bias=True), torch.float16, 44, layout,
+                    algo="dense_tc", expect_kernel="dense_tc")

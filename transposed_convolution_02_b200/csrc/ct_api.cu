@@ -38,7 +38,7 @@ ct_status resolve(const ct_desc *d, Plan *p) {
     if (d->dtype != CT_F32 && d->dtype != CT_F16) return CT_ERR_DTYPE;
     if (d->layout != CT_NCHW && d->layout != CT_NHWC) return CT_ERR_DTYPE;
     if (d->auto_pad < CT_AUTOPAD_NOTSET || d->auto_pad > CT_AUTOPAD_VALID) return CT_ERR_ATTR;
-    if (d->algo < CT_ALGO_AUTO || d->algo > CT_ALGO_GROUPED) return CT_ERR_ATTR;
+    if (d->algo < CT_ALGO_AUTO || d->algo > CT_ALGO_DENSE_TC_PERTAP) return CT_ERR_ATTR;
     const int r = d->rank;
     if (d->N < 0 || d->C < 0) return CT_ERR_ATTR;
     if (d->group <= 0 || d->C % d->group != 0) return CT_ERR_CHANNELS;
@@ -143,6 +143,9 @@ void choose(Plan *p) {
     if (want == CT_ALGO_GENERIC) return;
     if ((want == CT_ALGO_AUTO || want == CT_ALGO_DENSE_TC) && dense_tc_supports(*p)) {
         p->algo = CT_ALGO_DENSE_TC;
+    } else if ((want == CT_ALGO_AUTO || want == CT_ALGO_DENSE_TC || want == CT_ALGO_DENSE_TC_PERTAP) &&
+               dense_pertap_supports(*p)) {
+        p->algo = CT_ALGO_DENSE_TC_PERTAP;
     } else if ((want == CT_ALGO_AUTO || want == CT_ALGO_GROUPED) && grouped_supports(*p)) {
         p->algo = CT_ALGO_GROUPED;
     } else if ((want == CT_ALGO_AUTO || want == CT_ALGO_FP32_GEMM) && fp32_gemm_supports(*p)) {
@@ -231,6 +234,11 @@ ct_status ct_plan(const ct_desc *desc, ct_plan_t **out) {
             p->packed_bytes = dense_tc_packed_bytes(*p);
             p->ws_bytes = dense_tc_ws_bytes(*p);
             break;
+        case CT_ALGO_DENSE_TC_PERTAP:
+            dense_pertap_setup(*p);
+            p->packed_bytes = dense_pertap_packed_bytes(*p);
+            p->ws_bytes = dense_pertap_ws_bytes(*p);
+            break;
         case CT_ALGO_GROUPED: p->packed_bytes = grouped_packed_bytes(*p); break;
         case CT_ALGO_FP32_GEMM: p->packed_bytes = fp32_gemm_packed_bytes(*p); break;
         default: p->packed_bytes = generic_packed_bytes(*p); break;
@@ -243,6 +251,7 @@ const char *ct_plan_kernel(const ct_plan_t *plan) {
     if (!plan) return "";
     switch (reinterpret_cast<const Plan *>(plan)->algo) {
         case CT_ALGO_DENSE_TC: return "dense_tc";
+        case CT_ALGO_DENSE_TC_PERTAP: return "dense_tc_pertap";
         case CT_ALGO_FP32_GEMM: return "fp32_gemm";
         case CT_ALGO_GROUPED: return "grouped";
         default: return "generic";
@@ -278,6 +287,7 @@ ct_status ct_prepack_weights(const ct_plan_t *plan, const void *w, void *w_packe
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     switch (p.algo) {
         case CT_ALGO_DENSE_TC: return dense_tc_prepack(p, w, w_packed, s);
+        case CT_ALGO_DENSE_TC_PERTAP: return dense_pertap_prepack(p, w, w_packed, s);
         case CT_ALGO_GROUPED: return grouped_prepack(p, w, w_packed, s);
         case CT_ALGO_FP32_GEMM: return fp32_gemm_prepack(p, w, w_packed, s);
         default: return generic_prepack(p, w, w_packed, s);
@@ -308,6 +318,7 @@ ct_status ct_run(const ct_plan_t *plan, const void *x, const void *w_packed, con
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     switch (p.algo) {
         case CT_ALGO_DENSE_TC: return dense_tc_run(p, x, w_packed, bias, y, workspace, s);
+        case CT_ALGO_DENSE_TC_PERTAP: return dense_pertap_run(p, x, w_packed, bias, y, workspace, s);
         case CT_ALGO_GROUPED: return grouped_run(p, x, w_packed, bias, y, s);
         case CT_ALGO_FP32_GEMM: return fp32_gemm_run(p, x, w_packed, bias, y, s);
         default: return generic_run(p, x, w_packed, bias, y, s);

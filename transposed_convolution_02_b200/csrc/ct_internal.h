@@ -57,6 +57,19 @@ ct_status generic_prepack(const Plan &p, const void *w, void *wp, cudaStream_t s
 ct_status generic_run(const Plan &p, const void *x, const void *wp, const void *bias, void *y,
                       cudaStream_t st);
 
+// shared layout helpers (k_relayout.cu)
+ct_status launch_nchw_to_nhwc_f16(const Plan &p, const void *x, void *xt, cudaStream_t st);
+bool has_dead_phases(const Plan &p);
+ct_status launch_dead_fill(const Plan &p, const void *bias, void *y, cudaStream_t st);
+
+bool dense_pertap_supports(const Plan &p);
+size_t dense_pertap_packed_bytes(const Plan &p);
+size_t dense_pertap_ws_bytes(const Plan &p);
+void dense_pertap_setup(Plan &p);
+ct_status dense_pertap_prepack(const Plan &p, const void *w, void *wp, cudaStream_t st);
+ct_status dense_pertap_run(const Plan &p, const void *x, const void *wp, const void *bias, void *y,
+                           void *ws, cudaStream_t st);
+
 bool dense_tc_supports(const Plan &p);
 size_t dense_tc_packed_bytes(const Plan &p);
 size_t dense_tc_ws_bytes(const Plan &p);

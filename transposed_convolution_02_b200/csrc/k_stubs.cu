@@ -2,12 +2,6 @@
 #include "ct_internal.h"
 
 namespace ct {
-bool dense_tc_supports(const Plan &) { return false; }
-size_t dense_tc_packed_bytes(const Plan &) { return 0; }
-size_t dense_tc_ws_bytes(const Plan &) { return 0; }
-void dense_tc_setup(Plan &) {}
-ct_status dense_tc_prepack(const Plan &, const void *, void *, cudaStream_t) { return CT_ERR_UNSUPPORTED; }
-ct_status dense_tc_run(const Plan &, const void *, const void *, const void *, void *, void *, cudaStream_t) { return CT_ERR_UNSUPPORTED; }
 bool fp32_gemm_supports(const Plan &) { return false; }
 size_t fp32_gemm_packed_bytes(const Plan &) { return 0; }
 ct_status fp32_gemm_prepack(const Plan &, const void *, void *, cudaStream_t) { return CT_ERR_UNSUPPORTED; }
