@@ -158,6 +158,27 @@ CT_API ct_status ct_prepack_weights(const ct_plan_t *plan, const void *w, void *
 CT_API ct_status ct_run(const ct_plan_t *plan, const void *x, const void *w_packed,
                  const void *bias, void *y, void *workspace, void *stream);
 
+/* Size of the device array that ct_run_noalloc uses as its workspace.  Every
+ * GPU that loads libct.so holds this much device memory until the process
+ * exits. */
+#define CT_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+/* ct_run for callers that cannot allocate device memory while running, such
+ * as a plugin inside an engine that owns all device memory, or a loop whose
+ * rules forbid allocation after start-up.  The ONNX page and the ClikaRT page
+ * have no counterpart of this call; it exists only for such callers.  The
+ * caller still passes x, w_packed, bias and y as for ct_run.  The workspace
+ * comes from a fixed array of CT_NOALLOC_SCRATCH_BYTES inside the library:
+ * plans whose ct_workspace_bytes exceed that return CT_ERR_WORKSPACE.  The
+ * first call on a device that needs the array looks up its device address on
+ * the current device; make that first call before any stream capture.  No
+ * call allocates device memory.  All calls share the one array (it keeps the
+ * last call's contents; the kernels overwrite all workspace bytes they read),
+ * so calls whose GPU work overlaps in time, for example on two streams,
+ * race on it and must be serialised by the caller. */
+CT_API ct_status ct_run_noalloc(const ct_plan_t *plan, const void *x, const void *w_packed,
+                                const void *bias, void *y, void *stream);
+
 CT_API void ct_plan_destroy(ct_plan_t *plan);
 
 /* Static, human-readable text for a status code. */

@@ -15,6 +15,7 @@ from .ct import (  # noqa: F401
     ct_prepack_weights,
     ct_prepacked_weight_bytes,
     ct_run,
+    ct_run_noalloc,
     ct_status_string,
     ct_workspace_bytes,
     make_desc,

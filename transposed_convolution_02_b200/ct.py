@@ -32,8 +32,8 @@ ALGO = {"auto": 0, "generic": 1, "dense_tc": 2, "fp32_gemm": 3, "grouped": 4,
 
 EXPORTED = ["ct_output_shape", "ct_plan", "ct_plan_kernel", "ct_plan_launches",
             "ct_prepacked_weight_bytes",
-            "ct_workspace_bytes", "ct_prepack_weights", "ct_run", "ct_plan_destroy",
-            "ct_status_string"]
+            "ct_workspace_bytes", "ct_prepack_weights", "ct_run", "ct_run_noalloc",
+            "ct_plan_destroy", "ct_status_string"]
 
 
 class CtError(RuntimeError):
@@ -80,12 +80,13 @@ def lib():
         L.ct_workspace_bytes.argtypes = [P, szp]
         L.ct_prepack_weights.argtypes = [P, P, P, P]
         L.ct_run.argtypes = [P, P, P, P, P, P, P]
+        L.ct_run_noalloc.argtypes = [P, P, P, P, P, P]
         L.ct_plan_destroy.argtypes = [P]
         L.ct_plan_destroy.restype = None
         L.ct_status_string.argtypes = [ctypes.c_int]
         L.ct_status_string.restype = ctypes.c_char_p
         for name in ("ct_output_shape", "ct_plan", "ct_plan_launches", "ct_prepacked_weight_bytes",
-                     "ct_workspace_bytes", "ct_prepack_weights", "ct_run"):
+                     "ct_workspace_bytes", "ct_prepack_weights", "ct_run", "ct_run_noalloc"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -154,6 +155,14 @@ def ct_run(plan, x_ptr, wp_ptr, bias_ptr, y_ptr, ws_ptr, stream):
     st = lib().ct_run(plan, x_ptr, wp_ptr, bias_ptr, y_ptr, ws_ptr, stream)
     if st != CT_OK:
         raise CtError(st, "ct_run")
+
+
+def ct_run_noalloc(plan, x_ptr, wp_ptr, bias_ptr, y_ptr, stream):
+    """ct_run with the workspace taken from the library's fixed device array
+    (for callers that may not allocate device memory while running)."""
+    st = lib().ct_run_noalloc(plan, x_ptr, wp_ptr, bias_ptr, y_ptr, stream)
+    if st != CT_OK:
+        raise CtError(st, "ct_run_noalloc")
 
 
 def ct_plan_destroy(plan):
