@@ -9,19 +9,24 @@
 // channels on its N side, the reduction runs over (input channel, tap).
 //
 // Reuse:
-//  * One TMA tile per (x-offset, z-offset, 64-channel block) holds the input
-//    rows a whole unit needs plus the y halo; every tap with that x/z offset
-//    reads it through a descriptor shifted by whole J-rows (a multiple of
-//    1024 bytes, so the 128-byte swizzle phase is unchanged).
+//  * A unit's input is ONE TMA tile per 64-channel block: a box of HX x HYb x
+//    HZb input pixels (the unit's pixels plus the halo every tap needs), each
+//    pixel a 128-byte row of 64 channels in the 128-byte-swizzled K-major
+//    layout.  The unit's output pixels are numbered in the same pitch (HX
+//    per row), so every tap is the same 128 rows shifted by a constant; the
+//    MMA descriptor simply starts at that row (the swizzle follows the
+//    absolute shared address, so any 128-byte row start is valid).  Lanes
+//    that fall on halo columns compute values that are never stored.
 //  * (phase, tap) pairs with the same input offset whose phases own adjacent
 //    TMEM accumulators run as one MMA with a wider N.
-//  * A unit covers Mt tiles of 128 pixels, so each weight tile feeds Mt MMAs;
-//    weights stay resident in shared memory when the whole packed weight fits.
+//  * A unit covers Mt tiles of 128 positions, so each weight tile feeds Mt
+//    MMAs; weights stay resident in shared memory when they all fit.
 // Warps: 0 loads input tiles, 1 issues MMAs, 2 loads weights, 4-7 drain TMEM
 // (bias from shared memory, fp16 rounding, paired x phases stored as half2).
 #include <cuda.h>
 
 #include <algorithm>
+#include <array>
 #include <atomic>
 #include <vector>
 
@@ -33,40 +38,36 @@ namespace ct {
 namespace {
 
 constexpr int kMaxPhases = 64;
-constexpr int kMaxGroups = 32;
-constexpr int kMaxClasses = 64;
-constexpr int kMaxItems = 320;
+constexpr int kMaxGroups = 64;
+constexpr int kMaxItems = 512;
 constexpr int kThreads = 256;
 constexpr int kSmemBudget = 227 * 1024;
 
 struct Item {
     int16_t e[3];       // input offset (z, y, x)
-    int16_t row_shift;  // pixel rows into the class's input tile
     int16_t n;          // MMA N: run length x Np
+    int32_t shift;      // rows from a position to its input under this offset
     int16_t tcol;       // first TMEM column of the run inside the group
     int16_t phase0;     // first phase of the run (global live-phase index)
     int16_t first;      // first write of these columns (at channel block 0)
+    int16_t pad;
     int32_t brow;       // row offset of this item's weights inside one channel block
-};
-
-struct Class {
-    int16_t ex, ez, ey_min, item0, nitems, pad;
 };
 
 struct HaloTables {
     int32_t N, C, M, Np, KB;
     int32_t out[3], s[3], nJ[3], pb[3], d[3], k[3];
-    int32_t BX, R, Mt, BYh;
-    int32_t TX, TY, TZ, n_units, n_groups;
-    int32_t nbuf, bufcols, SA, SB, a_bytes, b_slot_bytes, BR;
+    int32_t emin[3], span[3];
+    int32_t BXt, HX, HYb, HZb, Mt;      // x-tile width, input-tile box, M-tiles per unit
+    int32_t TX, PU, n_units, n_groups;  // x tiles, units per (n, z, x-tile) plane
+    int32_t nbuf, bufcols, SA, SB, a_bytes, a_stride, b_slot_bytes, BR;
     int32_t resident, res_rows;
     int32_t nhwc, has_bias, dead, pair_x;
-    int32_t n_phases, n_items, n_classes;
-    int32_t total_rows;
+    int32_t n_phases, n_items, total_rows;
     int16_t phase_r[kMaxPhases][3];
-    int16_t g_phase0[kMaxGroups], g_nphase[kMaxGroups], g_cls0[kMaxGroups], g_ncls[kMaxGroups];
+    int16_t g_phase0[kMaxGroups], g_nphase[kMaxGroups], g_item0[kMaxGroups], g_nitem[kMaxGroups];
+    int16_t g_emin[kMaxGroups][3];      // smallest input offset of the group's taps
     int32_t g_brow[kMaxGroups], g_rows_kb[kMaxGroups];
-    Class cls[kMaxClasses];
     Item item[kMaxItems];
 };
 
@@ -89,15 +90,13 @@ __global__ void __launch_bounds__(256) halo_prepack_kernel(const __grid_constant
          i += (long long)gridDim.x * blockDim.x) {
         const int cc = (int)(i & 63);
         const int row = (int)(i >> 6);
-        // find the group, channel block and item of this row
         int g = 0;
         while (g + 1 < T.n_groups && row >= T.g_brow[g + 1]) ++g;
         const int rg = row - T.g_brow[g];
         const int kb = rg / T.g_rows_kb[g];
         const int rk = rg % T.g_rows_kb[g];
-        const int i0 = T.cls[T.g_cls0[g]].item0;
-        const int i1 = T.cls[T.g_cls0[g] + T.g_ncls[g] - 1].item0 + T.cls[T.g_cls0[g] + T.g_ncls[g] - 1].nitems;
-        int it = i0;
+        int it = T.g_item0[g];
+        const int i1 = T.g_item0[g] + T.g_nitem[g];
         while (it + 1 < i1 && rk >= T.item[it + 1].brow) ++it;
         const Item &I = T.item[it];
         const int rr = rk - I.brow;
@@ -123,20 +122,59 @@ __global__ void __launch_bounds__(256) halo_prepack_kernel(const __grid_constant
 }
 
 // ---------------------------------------------------------------------------
+// A unit: image n, output z-slice jz, x-tile tx, positions [F0, F0 + Mt*128)
+// of the (y, x) plane numbered f = jy * HX + jx (jx < BXt valid), group g.
+// The kernel copies every table it walks into shared memory and every scalar
+// into registers at start: the parameter block is large, and re-reading it
+// between the tcgen05 instructions costs constant-cache misses.
 
-struct Unit {
-    int g, n, tz, ty, tx;
+struct SItem {
+    int32_t shift;
+    int32_t brow;
+    int16_t n, tcol, first, pad;
+};
+struct SGroup {
+    int32_t brow, rows_kb;
+    int16_t item0, nitem, phase0, nphase;
+    int16_t emin[3], pad;
 };
 
-__device__ __forceinline__ Unit decode_unit(const HaloTables &T, int u) {
+struct Geo {
+    int n_groups, PU, TX, nJz, Mt, HX;
+};
+
+struct Unit {
+    int g, n, jz, tx, F0, y0;
+};
+
+__device__ __forceinline__ Unit decode_unit(const Geo &G, int u) {
     Unit r;
-    r.g = u % T.n_groups;
-    int t = u / T.n_groups;
-    r.tx = t % T.TX; t /= T.TX;
-    r.ty = t % T.TY; t /= T.TY;
-    r.tz = t % T.TZ;
-    r.n = t / T.TZ;
+    r.g = u % G.n_groups;
+    int t = u / G.n_groups;
+    const int pu = t % G.PU;
+    t /= G.PU;
+    r.tx = t % G.TX;
+    t /= G.TX;
+    r.jz = t % G.nJz;
+    r.n = t / G.nJz;
+    r.F0 = pu * G.Mt * 128;
+    r.y0 = r.F0 / G.HX;
     return r;
+}
+
+// The four K = 16 steps of one 64-channel block (descriptor start + 32 bytes each).
+__device__ __forceinline__ void issue4(uint32_t d, uint64_t ad, uint64_t bd, uint32_t idesc, uint32_t acc0) {
+    sm100::mma_f16(d, ad, bd, idesc, acc0);
+    sm100::mma_f16(d, ad + 2, bd + 2, idesc, 1u);
+    sm100::mma_f16(d, ad + 4, bd + 4, idesc, 1u);
+    sm100::mma_f16(d, ad + 6, bd + 6, idesc, 1u);
+}
+
+__device__ __forceinline__ void store_chunk16(__half *dst, long long stride, const uint32_t (&v)[16],
+                                              const float *b, int mcount) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+        if (j < mcount) dst[j * stride] = __float2half_rn(__uint_as_float(v[j]) + b[j]);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -147,12 +185,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int SA = T.SA, SB = T.SB;
+    // scalars in registers
+    const int SA = T.SA, SB = T.SB, KB = T.KB, Np = T.Np, M = T.M, Mt = T.Mt;
+    const int n_units = T.n_units, resident = T.resident, nbuf = T.nbuf, bufcols = T.bufcols;
+    const int a_stride = T.a_stride, a_bytes = T.a_bytes, b_slot = T.b_slot_bytes, BR = T.BR;
+    const int res_rows = T.res_rows, BXt = T.BXt, HX = T.HX, nhwc = T.nhwc, pair_x = T.pair_x;
+    const int n_items = T.n_items, n_groups = T.n_groups, n_phases = T.n_phases;
+    const Geo G{T.n_groups, T.PU, T.TX, T.nJ[0], T.Mt, T.HX};
+    // shared-memory layout
     uint8_t *sA = smem;
-    uint8_t *sB = sA + (size_t)SA * T.a_bytes;       // ring slots, or the resident weights
-    const size_t b_region = T.resident ? (size_t)T.res_rows * 128 : (size_t)SB * T.b_slot_bytes;
+    uint8_t *sB = sA + (size_t)SA * a_stride;       // ring slots, or the resident weights
+    const size_t b_region = resident ? (size_t)res_rows * 128 : (size_t)SB * b_slot;
     float *bias_s = reinterpret_cast<float *>(sB + b_region);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(bias_s + T.Np);
+    SItem *items_s = reinterpret_cast<SItem *>(bias_s + Np);
+    SGroup *groups_s = reinterpret_cast<SGroup *>(items_s + n_items);
+    int16_t *phr_s = reinterpret_cast<int16_t *>(groups_s + n_groups);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(((uintptr_t)(phr_s + 3 * n_phases) + 7) & ~(uintptr_t)7);
     const uint32_t fullA = smem_u32(bars), emptyA = smem_u32(bars + SA);
     const uint32_t fullB = smem_u32(bars + 2 * SA), emptyB = smem_u32(bars + 2 * SA + SB);
     const uint32_t tfull = smem_u32(bars + 2 * SA + 2 * SB);
@@ -180,10 +228,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tmap(&tmA);
         prefetch_tmap(&tmB);
     }
-    if (warp >= 4) {
-        for (int m = threadIdx.x - 128; m < T.Np; m += 128)
-            bias_s[m] = (T.has_bias && m < T.M) ? __half2float(bias[m]) : 0.f;
+    for (int i = threadIdx.x; i < n_items; i += kThreads) {
+        SItem it;
+        it.shift = T.item[i].shift;
+        it.brow = T.item[i].brow;
+        it.n = T.item[i].n;
+        it.tcol = T.item[i].tcol;
+        it.first = T.item[i].first;
+        it.pad = 0;
+        items_s[i] = it;
     }
+    for (int g = threadIdx.x; g < n_groups; g += kThreads) {
+        SGroup gr;
+        gr.brow = T.g_brow[g];
+        gr.rows_kb = T.g_rows_kb[g];
+        gr.item0 = T.g_item0[g];
+        gr.nitem = T.g_nitem[g];
+        gr.phase0 = T.g_phase0[g];
+        gr.nphase = T.g_nphase[g];
+        gr.emin[0] = T.g_emin[g][0];
+        gr.emin[1] = T.g_emin[g][1];
+        gr.emin[2] = T.g_emin[g][2];
+        gr.pad = 0;
+        groups_s[g] = gr;
+    }
+    for (int i = threadIdx.x; i < 3 * n_phases; i += kThreads) phr_s[i] = T.phase_r[i / 3][i % 3];
+    for (int m = threadIdx.x; m < Np; m += kThreads)
+        bias_s[m] = (T.has_bias && m < M) ? __half2float(bias[m]) : 0.f;
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_slot), 512);
         tmem_relinquish();
@@ -197,52 +268,49 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---------------- input tiles ----------------
         int ia = 0;
         bool ok = true;
-        for (int u = blockIdx.x; u < T.n_units && ok; u += gridDim.x) {
-            const Unit U = decode_unit(T, u);
-            const int J0x = U.tx * T.BX, J0y = U.ty * T.Mt * T.R, J0z = U.tz;
-            for (int kb = 0; kb < T.KB && ok; ++kb) {
-                for (int c = T.g_cls0[U.g]; c < T.g_cls0[U.g] + T.g_ncls[U.g]; ++c, ++ia) {
-                    const int s = ia % SA;
-                    if (ia >= SA && !mbar_wait(emptyA + 8 * s, ((ia / SA) - 1) & 1, err, 1)) {
-                        ok = false;
-                        break;
-                    }
-                    mbar_arrive_expect_tx(fullA + 8 * s, T.a_bytes);
-                    tma_load_5d(smem_u32(sA + (size_t)s * T.a_bytes), &tmA, fullA + 8 * s, kb * 64,
-                                J0x + T.cls[c].ex, J0y + T.cls[c].ey_min, J0z + T.cls[c].ez, U.n);
+        for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+            const Unit U = decode_unit(G, u);
+            const SGroup gr = groups_s[U.g];
+            const int x0 = U.tx * BXt + gr.emin[2];
+            const int y0 = U.y0 + gr.emin[1];
+            const int z0 = U.jz + gr.emin[0];
+            for (int kb = 0; kb < KB; ++kb, ++ia) {
+                const int s = ia % SA;
+                if (ia >= SA && !mbar_wait(emptyA + 8 * s, ((ia / SA) - 1) & 1, err, 1)) {
+                    ok = false;
+                    break;
                 }
+                mbar_arrive_expect_tx(fullA + 8 * s, a_bytes);
+                tma_load_5d(smem_u32(sA + (size_t)s * a_stride), &tmA, fullA + 8 * s, kb * 64, x0, y0, z0, U.n);
             }
         }
         const int first = ia > SA ? ia - SA : 0;
         for (int j = first; j < ia; ++j) mbar_wait(fullA + 8 * (j % SA), (j / SA) & 1, err, 2);
     } else if (warp == 2 && lane == 0) {
         // ---------------- weight tiles ----------------
-        if (T.resident) {
-            mbar_arrive_expect_tx(bres, (uint32_t)T.res_rows * 128);
-            for (int r = 0; r < T.res_rows; r += T.BR)
-                tma_load_2d(smem_u32(sB + (size_t)r * 128), &tmB, bres, 0, r);
+        if (resident) {
+            mbar_arrive_expect_tx(bres, (uint32_t)res_rows * 128);
+            for (int r = 0; r < res_rows; r += BR) tma_load_2d(smem_u32(sB + (size_t)r * 128), &tmB, bres, 0, r);
             mbar_wait(bres, 0, err, 3);
         } else {
             int ib = 0;
             bool ok = true;
-            for (int u = blockIdx.x; u < T.n_units && ok; u += gridDim.x) {
-                const Unit U = decode_unit(T, u);
-                for (int kb = 0; kb < T.KB && ok; ++kb) {
-                    const int c0 = T.g_cls0[U.g];
-                    const int i0 = T.cls[c0].item0;
-                    const int i1 = T.cls[c0 + T.g_ncls[U.g] - 1].item0 + T.cls[c0 + T.g_ncls[U.g] - 1].nitems;
-                    const int rowbase = T.g_brow[U.g] + kb * T.g_rows_kb[U.g];
-                    for (int it = i0; it < i1; ++it, ++ib) {
+            for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+                const Unit U = decode_unit(G, u);
+                const SGroup gr = groups_s[U.g];
+                for (int kb = 0; kb < KB && ok; ++kb) {
+                    const int rowbase = gr.brow + kb * gr.rows_kb;
+                    for (int it = gr.item0; it < gr.item0 + gr.nitem; ++it, ++ib) {
                         const int s = ib % SB;
                         if (ib >= SB && !mbar_wait(emptyB + 8 * s, ((ib / SB) - 1) & 1, err, 4)) {
                             ok = false;
                             break;
                         }
-                        const int n = T.item[it].n;
-                        mbar_arrive_expect_tx(fullB + 8 * s, (uint32_t)n * 128);
-                        for (int r = 0; r < n; r += T.BR)
-                            tma_load_2d(smem_u32(sB + (size_t)s * T.b_slot_bytes + (size_t)r * 128), &tmB,
-                                        fullB + 8 * s, 0, rowbase + T.item[it].brow + r);
+                        const SItem I = items_s[it];
+                        mbar_arrive_expect_tx(fullB + 8 * s, (uint32_t)I.n * 128);
+                        for (int r = 0; r < I.n; r += BR)
+                            tma_load_2d(smem_u32(sB + (size_t)s * b_slot + (size_t)r * 128), &tmB, fullB + 8 * s, 0,
+                                        rowbase + I.brow + r);
                     }
                 }
             }
@@ -252,58 +320,62 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1 && lane == 0) {
         // ---------------- MMA issue ----------------
         bool ok = true;
-        if (T.resident) ok = mbar_wait(bres, 0, err, 6);
+        if (resident) ok = mbar_wait(bres, 0, err, 6);
         int ia = 0, ib = 0, local = 0;
-        for (int u = blockIdx.x; u < T.n_units && ok; u += gridDim.x, ++local) {
-            const Unit U = decode_unit(T, u);
-            const int buf = T.nbuf == 2 ? (local & 1) : 0;
-            const int use = T.nbuf == 2 ? (local >> 1) : local;
+        for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++local) {
+            const Unit U = decode_unit(G, u);
+            const SGroup gr = groups_s[U.g];
+            const int buf = nbuf == 2 ? (local & 1) : 0;
+            const int use = nbuf == 2 ? (local >> 1) : local;
             if (use > 0 && !mbar_wait(tempty + 8 * buf, (use - 1) & 1, err, 7)) break;
             tc_fence_after();
-            const uint32_t dbase = tmem_base + buf * T.bufcols;
-            const int gcols = T.g_nphase[U.g] * T.Np;
-            for (int kb = 0; kb < T.KB && ok; ++kb) {
-                for (int c = T.g_cls0[U.g]; c < T.g_cls0[U.g] + T.g_ncls[U.g] && ok; ++c, ++ia) {
-                    const int sa = ia % SA;
-                    if (!mbar_wait(fullA + 8 * sa, (ia / SA) & 1, err, 8)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t a_addr = smem_u32(sA + (size_t)sa * T.a_bytes);
-                    for (int it = T.cls[c].item0; it < T.cls[c].item0 + T.cls[c].nitems; ++it) {
-                        const Item &I = T.item[it];
-                        uint32_t b_addr;
-                        int sb = 0;
-                        if (T.resident) {
-                            b_addr = smem_u32(sB) + (uint32_t)((kb * T.g_rows_kb[U.g] + I.brow) * 128);
-                        } else {
-                            sb = ib % SB;
-                            if (!mbar_wait(fullB + 8 * sb, (ib / SB) & 1, err, 9)) {
-                                ok = false;
-                                break;
-                            }
-                            tc_fence_after();
-                            b_addr = smem_u32(sB + (size_t)sb * T.b_slot_bytes);
-                        }
-                        const uint32_t idesc = idesc_f16_f32(128, I.n);
-                        const uint64_t bd = desc_kmajor_sw128(b_addr);
-                        const uint32_t acc0 = (kb == 0 && I.first) ? 0u : 1u;
-                        for (int mt = 0; mt < T.Mt; ++mt) {
-                            const uint64_t ad =
-                                desc_kmajor_sw128(a_addr + (uint32_t)((I.row_shift + mt * 128) * 128));
-                            const uint32_t d = dbase + mt * gcols + I.tcol;
-#pragma unroll
-                            for (int kk = 0; kk < 4; ++kk)
-                                mma_f16(d, ad + 2 * kk, bd + 2 * kk, idesc, kk == 0 ? acc0 : 1u);
-                        }
-                        if (!T.resident) {
-                            mma_commit(emptyB + 8 * sb);
-                            ++ib;
-                        }
-                    }
-                    mma_commit(emptyA + 8 * sa);
+            const uint32_t dbase = tmem_base + buf * bufcols;
+            const int gcols = gr.nphase * Np;
+            const int rel = U.F0 - U.y0 * HX;   // row of the unit's first position in the tile
+            for (int kb = 0; kb < KB && ok; ++kb, ++ia) {
+                const int sa = ia % SA;
+                if (!mbar_wait(fullA + 8 * sa, (ia / SA) & 1, err, 8)) {
+                    ok = false;
+                    break;
                 }
+                tc_fence_after();
+                const uint32_t a_addr = smem_u32(sA + (size_t)sa * a_stride) + (uint32_t)rel * 128;
+                const uint32_t bres_base = smem_u32(sB) + (uint32_t)((gr.brow + kb * gr.rows_kb) * 128);
+                const int i0 = gr.item0, i1 = gr.item0 + gr.nitem;
+                const uint32_t mstep = (uint32_t)gcols;
+                if (resident) {
+                    // weights resident: nothing to wait for between items
+                    for (int it = i0; it < i1; ++it) {
+                        const SItem I = items_s[it];
+                        const uint64_t bd = desc_kmajor_sw128(bres_base + (uint32_t)I.brow * 128);
+                        const uint64_t ad = desc_kmajor_sw128(a_addr + (uint32_t)I.shift * 128);
+                        const uint32_t idesc = idesc_f16_f32(128, I.n);
+                        const uint32_t d = dbase + I.tcol;
+                        const uint32_t acc0 = (kb == 0 && I.first) ? 0u : 1u;
+                        issue4(d, ad, bd, idesc, acc0);
+                        if (Mt > 1) issue4(d + mstep, ad + 1024, bd, idesc, acc0);   // +128 rows
+                    }
+                } else {
+                    for (int it = i0; it < i1; ++it) {
+                        const SItem I = items_s[it];
+                        const int sb = ib % SB;
+                        if (!mbar_wait(fullB + 8 * sb, (ib / SB) & 1, err, 9)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint64_t bd = desc_kmajor_sw128(smem_u32(sB + (size_t)sb * b_slot));
+                        const uint64_t ad = desc_kmajor_sw128(a_addr + (uint32_t)I.shift * 128);
+                        const uint32_t idesc = idesc_f16_f32(128, I.n);
+                        const uint32_t d = dbase + I.tcol;
+                        const uint32_t acc0 = (kb == 0 && I.first) ? 0u : 1u;
+                        issue4(d, ad, bd, idesc, acc0);
+                        if (Mt > 1) issue4(d + mstep, ad + 1024, bd, idesc, acc0);   // +128 rows
+                        mma_commit(emptyB + 8 * sb);
+                        ++ib;
+                    }
+                }
+                mma_commit(emptyA + 8 * sa);
             }
             mma_commit(tfull + 8 * buf);
         }
@@ -313,79 +385,77 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---------------- epilogue ----------------
         const int lane_base = 32 * (warp & 3);
         const int p = lane_base + lane;
-        const long long plane = (long long)T.out[0] * T.out[1] * T.out[2];
+        const int out0 = T.out[0], out1 = T.out[1], out2 = T.out[2];
+        const int s0 = T.s[0], s1 = T.s[1], s2 = T.s[2];
+        const int nJ1 = T.nJ[1], nJ2 = T.nJ[2];
+        const long long plane = (long long)out0 * out1 * out2;
+        const long long cstride = nhwc ? 1 : plane;        // between channels
+        const long long xstep = nhwc ? (long long)M : 1;   // between x positions
         int local = 0;
-        for (int u = blockIdx.x; u < T.n_units; u += gridDim.x, ++local) {
-            const Unit U = decode_unit(T, u);
-            const int buf = T.nbuf == 2 ? (local & 1) : 0;
-            const int use = T.nbuf == 2 ? (local >> 1) : local;
+        for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++local) {
+            const Unit U = decode_unit(G, u);
+            const SGroup gr = groups_s[U.g];
+            const int buf = nbuf == 2 ? (local & 1) : 0;
+            const int use = nbuf == 2 ? (local >> 1) : local;
             if (!mbar_wait(tfull + 8 * buf, use & 1, err, 11)) break;
             tc_fence_after();
-            const uint32_t dbase = tmem_base + ((uint32_t)lane_base << 16) + buf * T.bufcols;
-            const int gcols = T.g_nphase[U.g] * T.Np;
-            const int ph0 = T.g_phase0[U.g], ph1 = ph0 + T.g_nphase[U.g];
-            const int Jx = U.tx * T.BX + (p % T.BX);
-            const int Jz = U.tz;
-            for (int mt = 0; mt < T.Mt; ++mt) {
-                const int Jy = U.ty * T.Mt * T.R + mt * T.R + p / T.BX;
+            const uint32_t dbase = tmem_base + ((uint32_t)lane_base << 16) + buf * bufcols;
+            const int gcols = gr.nphase * Np;
+            const int ph0 = gr.phase0, ph1 = ph0 + gr.nphase;
+            for (int mt = 0; mt < Mt; ++mt) {
+                const int F = U.F0 + mt * 128 + p;
+                const int jxl = F % HX;
+                const int Jy = F / HX;
+                const int Jx = U.tx * BXt + jxl;
+                const bool pos_ok = jxl < BXt && Jx < nJ2 && Jy < nJ1;
                 for (int ph = ph0; ph < ph1;) {
-                    const int oz = T.s[0] * Jz + T.phase_r[ph][0];
-                    const int oy = T.s[1] * Jy + T.phase_r[ph][1];
-                    const int ox = T.s[2] * Jx + T.phase_r[ph][2];
-                    const bool valid = oz < T.out[0] && oy < T.out[1] && ox < T.out[2];
-                    const bool pair = T.pair_x && ph + 1 < ph1 && T.phase_r[ph][2] % 2 == 0 &&
-                                      T.phase_r[ph + 1][2] == T.phase_r[ph][2] + 1 &&
-                                      T.phase_r[ph + 1][1] == T.phase_r[ph][1] &&
-                                      T.phase_r[ph + 1][0] == T.phase_r[ph][0];
-                    const long long opos = ((long long)oz * T.out[1] + oy) * T.out[2] + ox;
-                    const uint32_t col0 = dbase + mt * gcols + (ph - ph0) * T.Np;
-                    for (int m0 = 0; m0 < T.Np; m0 += 16) {
-                        uint32_t v0[16], v1[16];
+                    const int r0 = phr_s[3 * ph], r1 = phr_s[3 * ph + 1], r2 = phr_s[3 * ph + 2];
+                    const int oz = s0 * U.jz + r0;
+                    const int oy = s1 * Jy + r1;
+                    const int ox = s2 * Jx + r2;
+                    const bool valid = pos_ok && oz < out0 && oy < out1 && ox < out2;
+                    const bool pair = pair_x && ph + 1 < ph1 && (r2 & 1) == 0 && phr_s[3 * ph + 5] == r2 + 1 &&
+                                      phr_s[3 * ph + 4] == r1 && phr_s[3 * ph + 3] == r0;
+                    const long long opos = ((long long)oz * out1 + oy) * out2 + ox;
+                    const uint32_t col0 = dbase + mt * gcols + (ph - ph0) * Np;
+                    __half *base = nhwc ? y + ((long long)U.n * plane + opos) * M : y + (long long)U.n * M * plane + opos;
+                    for (int m0 = 0; m0 < Np; m0 += 32) {
+                        uint32_t v0[16], v1[16], w0[16], w1[16];
+                        const bool two = m0 + 16 < Np;
                         tmem_ld16(col0 + m0, v0);
-                        if (pair) tmem_ld16(col0 + T.Np + m0, v1);
+                        if (two) tmem_ld16(col0 + m0 + 16, v1);
+                        if (pair) {
+                            tmem_ld16(col0 + Np + m0, w0);
+                            if (two) tmem_ld16(col0 + Np + m0 + 16, w1);
+                        }
                         tmem_ld_wait();
                         if (!valid) continue;
-                        if (T.nhwc) {
-                            __half *dst = y + ((long long)U.n * plane + opos) * T.M + m0;
-                            __align__(16) __half h[16];
+                        const int mc0 = min(16, M - m0), mc1 = min(16, M - m0 - 16);
+                        __half *dst = base + (long long)m0 * cstride;
+                        if (!nhwc && pair) {
+                            // both x phases of a channel are adjacent: one half2 per channel
 #pragma unroll
                             for (int j = 0; j < 16; ++j)
-                                h[j] = __float2half_rn(__uint_as_float(v0[j]) + bias_s[m0 + j]);
-                            if ((T.M & 7) == 0 && m0 + 16 <= T.M) {
-                                reinterpret_cast<uint4 *>(dst)[0] = reinterpret_cast<const uint4 *>(h)[0];
-                                reinterpret_cast<uint4 *>(dst)[1] = reinterpret_cast<const uint4 *>(h)[1];
-                            } else {
-                                for (int j = 0; j < 16 && m0 + j < T.M; ++j) dst[j] = h[j];
-                            }
-                            if (pair) {
-                                __half *dst1 = dst + T.M;   // x + 1
+                                if (j < mc0)
+                                    *reinterpret_cast<__half2 *>(dst + j * plane) =
+                                        __floats2half2_rn(__uint_as_float(v0[j]) + bias_s[m0 + j],
+                                                          __uint_as_float(w0[j]) + bias_s[m0 + j]);
+                            if (two) {
+                                __half *d1 = dst + 16 * plane;
 #pragma unroll
                                 for (int j = 0; j < 16; ++j)
-                                    h[j] = __float2half_rn(__uint_as_float(v1[j]) + bias_s[m0 + j]);
-                                if ((T.M & 7) == 0 && m0 + 16 <= T.M) {
-                                    reinterpret_cast<uint4 *>(dst1)[0] = reinterpret_cast<const uint4 *>(h)[0];
-                                    reinterpret_cast<uint4 *>(dst1)[1] = reinterpret_cast<const uint4 *>(h)[1];
-                                } else {
-                                    for (int j = 0; j < 16 && m0 + j < T.M; ++j) dst1[j] = h[j];
-                                }
+                                    if (j < mc1)
+                                        *reinterpret_cast<__half2 *>(d1 + j * plane) =
+                                            __floats2half2_rn(__uint_as_float(v1[j]) + bias_s[m0 + 16 + j],
+                                                              __uint_as_float(w1[j]) + bias_s[m0 + 16 + j]);
                             }
                         } else {
-                            __half *dst = y + ((long long)U.n * T.M + m0) * plane + opos;
+                            store_chunk16(dst, cstride, v0, bias_s + m0, mc0);
+                            if (two) store_chunk16(dst + 16 * cstride, cstride, v1, bias_s + m0 + 16, mc1);
                             if (pair) {
-#pragma unroll
-                                for (int j = 0; j < 16; ++j) {
-                                    if (m0 + j < T.M)
-                                        *reinterpret_cast<__half2 *>(dst + j * plane) =
-                                            __floats2half2_rn(__uint_as_float(v0[j]) + bias_s[m0 + j],
-                                                              __uint_as_float(v1[j]) + bias_s[m0 + j]);
-                                }
-                            } else {
-#pragma unroll
-                                for (int j = 0; j < 16; ++j) {
-                                    if (m0 + j < T.M)
-                                        dst[j * plane] =
-                                            __float2half_rn(__uint_as_float(v0[j]) + bias_s[m0 + j]);
-                                }
+                                __half *dx = dst + xstep;   // x + 1
+                                store_chunk16(dx, cstride, w0, bias_s + m0, mc0);
+                                if (two) store_chunk16(dx + 16 * cstride, cstride, w1, bias_s + m0 + 16, mc1);
                             }
                         }
                     }
@@ -405,19 +475,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 size_t smem_bytes(const HaloTables &T) {
     const size_t b_region = T.resident ? (size_t)T.res_rows * 128 : (size_t)T.SB * T.b_slot_bytes;
-    return 1024 + (size_t)T.SA * T.a_bytes + b_region + (size_t)T.Np * 4 +
+    const size_t tables = (size_t)T.n_items * sizeof(SItem) + (size_t)T.n_groups * sizeof(SGroup) +
+                          (size_t)T.n_phases * 6 + 8;
+    return 1024 + (size_t)T.SA * T.a_stride + b_region + (size_t)T.Np * 4 + tables +
            (size_t)(2 * T.SA + 2 * T.SB + 6) * 8 + 16;
 }
 
-int ilog2(int v) {
-    int l = 0;
-    while ((1 << l) < v) ++l;
-    return l;
-}
-
-// Build groups, classes and items for a given group policy.  Returns false if
-// a table limit is exceeded.
-bool build_tables(const Plan &p, HaloTables &T, int Mt_pref, bool single_row_groups) {
+// Build the tables for one policy: Mt M-tiles per unit and groups of at
+// most `gmax_cols` accumulator columns.  Returns false when a limit or the
+// shared-memory budget is exceeded.
+bool build_tables(const Plan &p, HaloTables &T, int Mt, int gmax_cols) {
     T.N = (int32_t)p.N;
     T.C = (int32_t)p.C;
     T.M = (int32_t)p.M;
@@ -425,6 +492,8 @@ bool build_tables(const Plan &p, HaloTables &T, int Mt_pref, bool single_row_gro
     T.KB = (int32_t)ceil_div(p.C, 64);
     T.nhwc = p.layout == CT_NHWC;
     T.has_bias = p.has_bias;
+    T.Mt = Mt;
+    if (T.Np > gmax_cols) return false;
     for (int a = 0; a < 3; ++a) {
         T.out[a] = (int32_t)p.out[a];
         T.s[a] = (int32_t)p.s[a];
@@ -434,9 +503,9 @@ bool build_tables(const Plan &p, HaloTables &T, int Mt_pref, bool single_row_gro
         T.k[a] = (int32_t)p.k[a];
     }
     T.pair_x = (p.s[2] % 2 == 0) && (p.out[2] % 2 == 0);
+    T.dead = has_dead_phases(p);
     // live phases
     int np = 0;
-    T.dead = has_dead_phases(p);
     for (int r0 = 0; r0 < p.s[0]; ++r0)
         for (int r1 = 0; r1 < p.s[1]; ++r1)
             for (int r2 = 0; r2 < p.s[2]; ++r2) {
@@ -449,8 +518,8 @@ bool build_tables(const Plan &p, HaloTables &T, int Mt_pref, bool single_row_gro
             }
     if (np == 0) return false;
     T.n_phases = np;
-    // groups: whole (r0, r1) rows of phases, merged while they fit 256 columns
-    const int per = 256 / T.Np;
+    // groups: whole (r0, r1) rows of phases, merged while within gmax_cols
+    const int per = gmax_cols / T.Np;
     auto same_row = [&](int a, int b) {
         return T.phase_r[a][0] == T.phase_r[b][0] && T.phase_r[a][1] == T.phase_r[b][1];
     };
@@ -460,7 +529,7 @@ bool build_tables(const Plan &p, HaloTables &T, int Mt_pref, bool single_row_gro
         while (end < np) {
             int row_end = end + 1;
             while (row_end < np && same_row(row_end, end)) ++row_end;
-            if (row_end - ph <= per && (!single_row_groups || end == ph))
+            if (row_end - ph <= per)
                 end = row_end;
             else
                 break;
@@ -476,8 +545,46 @@ bool build_tables(const Plan &p, HaloTables &T, int Mt_pref, bool single_row_gro
         ph = end;
     }
     T.n_groups = ng;
-    // classes and items per group
-    int nc = 0, ni = 0, rows_total = 0, span_max = 0;
+    // offset range of every group; the input tile is sized by the widest
+    for (int a = 0; a < 3; ++a) {
+        T.emin[a] = 0;
+        T.span[a] = 0;
+    }
+    for (int g = 0; g < ng; ++g) {
+        int lo[3] = {1 << 20, 1 << 20, 1 << 20}, hi[3] = {-(1 << 20), -(1 << 20), -(1 << 20)};
+        for (int ph = T.g_phase0[g]; ph < T.g_phase0[g] + T.g_nphase[g]; ++ph)
+            for (int a = 0; a < 3; ++a)
+                for (const Tap &t : p.taps[a][T.phase_r[ph][a]]) {
+                    lo[a] = std::min(lo[a], (int)t.e);
+                    hi[a] = std::max(hi[a], (int)t.e);
+                }
+        for (int a = 0; a < 3; ++a) {
+            T.g_emin[g][a] = (int16_t)lo[a];
+            T.span[a] = std::max(T.span[a], hi[a] - lo[a]);
+        }
+    }
+    // input tile geometry
+    if (T.nJ[2] + T.span[2] <= 256) {
+        T.BXt = T.nJ[2];
+    } else {
+        T.BXt = 256 - T.span[2];
+        if (T.BXt < 64) return false;
+    }
+    T.HX = T.BXt + T.span[2];
+    T.HYb = (int32_t)ceil_div((int64_t)Mt * 128 + T.HX + T.span[2], T.HX) + T.span[1];
+    T.HZb = 1 + T.span[0];
+    if (T.HYb > 256 || T.HZb > 256) return false;
+    T.a_bytes = T.HX * T.HYb * T.HZb * 128;
+    T.a_stride = (T.a_bytes + 1023) & ~1023;
+    T.TX = (int32_t)ceil_div(T.nJ[2], T.BXt);
+    const long long plane_pos = (long long)T.nJ[1] * T.HX;
+    T.PU = (int32_t)ceil_div(plane_pos, (long long)Mt * 128);
+    const long long units = (long long)T.N * T.nJ[0] * T.TX * T.PU * ng;
+    if (units > (1LL << 30)) return false;
+    T.n_units = (int32_t)units;
+    // items per group: pairs grouped by input offset, merged over adjacent phases
+    int ni = 0, rows_total = 0;
+    const int row_pitch = T.HX, slice_pitch = T.HX * T.HYb;
     for (int g = 0; g < ng; ++g) {
         struct PairRec { int ph, e0, e1, e2; };
         std::vector<PairRec> pairs;
@@ -487,96 +594,56 @@ bool build_tables(const Plan &p, HaloTables &T, int Mt_pref, bool single_row_gro
                 for (const Tap &b : p.taps[1][r1])
                     for (const Tap &c : p.taps[2][r2]) pairs.push_back({ph, a.e, b.e, c.e});
         }
-        // distinct (ez, ex) classes
-        std::vector<std::pair<int, int>> keys;
-        for (auto &q : pairs) keys.push_back({q.e0, q.e2});
-        std::sort(keys.begin(), keys.end());
-        keys.erase(std::unique(keys.begin(), keys.end()), keys.end());
-        T.g_cls0[g] = (int16_t)nc;
-        T.g_ncls[g] = (int16_t)keys.size();
+        std::vector<std::array<int, 3>> offs;
+        for (auto &q : pairs) offs.push_back({q.e0, q.e1, q.e2});
+        std::sort(offs.begin(), offs.end());
+        offs.erase(std::unique(offs.begin(), offs.end()), offs.end());
         std::vector<char> touched(np, 0);
+        T.g_item0[g] = (int16_t)ni;
         int brow = 0;
-        for (auto &kx : keys) {
-            if (nc >= kMaxClasses) return false;
-            Class &C = T.cls[nc];
-            C.ez = (int16_t)kx.first;
-            C.ex = (int16_t)kx.second;
-            std::vector<int> eys;
+        for (auto &e : offs) {
+            std::vector<int> phs;
             for (auto &q : pairs)
-                if (q.e0 == kx.first && q.e2 == kx.second) eys.push_back(q.e1);
-            std::sort(eys.begin(), eys.end());
-            eys.erase(std::unique(eys.begin(), eys.end()), eys.end());
-            C.ey_min = (int16_t)eys.front();
-            span_max = std::max(span_max, eys.back() - eys.front());
-            C.item0 = (int16_t)ni;
-            for (int ey : eys) {
-                std::vector<int> phs;
-                for (auto &q : pairs)
-                    if (q.e0 == kx.first && q.e2 == kx.second && q.e1 == ey) phs.push_back(q.ph);
-                std::sort(phs.begin(), phs.end());
-                // runs of consecutive phases with the same first-touch state, N <= 256
-                size_t i = 0;
-                while (i < phs.size()) {
-                    size_t j = i + 1;
-                    while (j < phs.size() && phs[j] == phs[j - 1] + 1 && touched[phs[j]] == touched[phs[i]] &&
-                           (int)(j - i + 1) * T.Np <= 256)
-                        ++j;
-                    if (ni >= kMaxItems) return false;
-                    Item &I = T.item[ni];
-                    I.e[0] = (int16_t)kx.first;
-                    I.e[1] = (int16_t)ey;
-                    I.e[2] = (int16_t)kx.second;
-                    I.row_shift = 0;   // set once BX is known
-                    I.n = (int16_t)((j - i) * T.Np);
-                    I.tcol = (int16_t)((phs[i] - T.g_phase0[g]) * T.Np);
-                    I.phase0 = (int16_t)phs[i];
-                    I.first = touched[phs[i]] ? 0 : 1;
-                    I.brow = brow;
-                    brow += I.n;
-                    for (size_t q = i; q < j; ++q) touched[phs[q]] = 1;
-                    ++ni;
-                    i = j;
-                }
+                if (q.e0 == e[0] && q.e1 == e[1] && q.e2 == e[2]) phs.push_back(q.ph);
+            std::sort(phs.begin(), phs.end());
+            size_t i = 0;
+            while (i < phs.size()) {
+                size_t j = i + 1;
+                while (j < phs.size() && phs[j] == phs[j - 1] + 1 && touched[phs[j]] == touched[phs[i]] &&
+                       (int)(j - i + 1) * T.Np <= 256)
+                    ++j;
+                if (ni >= kMaxItems) return false;
+                Item &I = T.item[ni];
+                I.e[0] = (int16_t)e[0];
+                I.e[1] = (int16_t)e[1];
+                I.e[2] = (int16_t)e[2];
+                I.n = (int16_t)((j - i) * T.Np);
+                I.shift = (e[0] - T.g_emin[g][0]) * slice_pitch + (e[1] - T.g_emin[g][1]) * row_pitch +
+                          (e[2] - T.g_emin[g][2]);
+                I.tcol = (int16_t)((phs[i] - T.g_phase0[g]) * T.Np);
+                I.phase0 = (int16_t)phs[i];
+                I.first = touched[phs[i]] ? 0 : 1;
+                I.pad = 0;
+                I.brow = brow;
+                brow += I.n;
+                for (size_t q = i; q < j; ++q) touched[phs[q]] = 1;
+                ++ni;
+                i = j;
             }
-            C.nitems = (int16_t)(ni - C.item0);
-            ++nc;
         }
+        T.g_nitem[g] = (int16_t)(ni - T.g_item0[g]);
         T.g_brow[g] = rows_total;
         T.g_rows_kb[g] = brow;
         rows_total += brow * T.KB;
     }
-    T.n_classes = nc;
     T.n_items = ni;
     T.total_rows = rows_total;
-    // tile geometry: BX J-columns (power of two, >= 8), R = 128 / BX J-rows per M-tile
-    int bx = 8;
-    while (bx < T.nJ[2] && bx < 128) bx *= 2;
-    T.BX = bx;
-    T.R = 128 / bx;
-    int mt = Mt_pref;
-    while (mt > 1 && (mt - 1) * T.R >= T.nJ[1]) --mt;   // no M-tile entirely past the rows
-    T.Mt = mt;
-    T.BYh = mt * T.R + span_max;
-    if (T.BYh > 256) return false;
-    for (int i = 0; i < ni; ++i) {
-        const Class *Cp = nullptr;
-        for (int c = 0; c < nc; ++c)
-            if (i >= T.cls[c].item0 && i < T.cls[c].item0 + T.cls[c].nitems) Cp = &T.cls[c];
-        T.item[i].row_shift = (int16_t)((T.item[i].e[1] - Cp->ey_min) * bx);
-    }
-    T.TX = (int32_t)ceil_div(T.nJ[2], bx);
-    T.TY = (int32_t)ceil_div(T.nJ[1], (int64_t)mt * T.R);
-    T.TZ = T.nJ[0];
-    const long long units = (long long)T.N * T.TZ * T.TY * T.TX * T.n_groups;
-    if (units > (1LL << 30)) return false;
-    T.n_units = (int32_t)units;
     // TMEM: Mt x group columns per buffer, double-buffered when that fits
-    int gmax = 0;
-    for (int g = 0; g < ng; ++g) gmax = std::max(gmax, (int)T.g_nphase[g] * T.Np);
-    T.bufcols = mt * gmax;
+    int gcols = 0;
+    for (int g = 0; g < ng; ++g) gcols = std::max(gcols, (int)T.g_nphase[g] * T.Np);
+    T.bufcols = Mt * gcols;
     if (T.bufcols > 512) return false;
     T.nbuf = T.bufcols <= 256 ? 2 : 1;
-    // weight box rows: largest power of two dividing every item N (<= 256)
     int br = 256;
     for (int i = 0; i < ni; ++i)
         while (T.item[i].n % br) br /= 2;
@@ -584,36 +651,63 @@ bool build_tables(const Plan &p, HaloTables &T, int Mt_pref, bool single_row_gro
     int nmax = 0;
     for (int i = 0; i < ni; ++i) nmax = std::max(nmax, (int)T.item[i].n);
     T.b_slot_bytes = nmax * 128;
-    T.a_bytes = bx * T.BYh * 128;
-    // shared memory: resident weights if the single group's packed rows fit
-    const int fixed = 1024 + T.Np * 4 + 64 * 8 + 64;
+    // shared memory: resident weights if they fit next to two input slots
+    const int fixed = 1024 + T.Np * 4 + 64 * 8 + 64 + ni * (int)sizeof(SItem) + ng * (int)sizeof(SGroup) +
+                      np * 6 + 8;
     T.resident = 0;
     T.res_rows = 0;
-    if (ng == 1 && (long long)rows_total * 128 + 3LL * T.a_bytes + fixed <= kSmemBudget) {
+    if ((long long)rows_total * 128 + 2LL * T.a_stride + fixed <= kSmemBudget) {
         T.resident = 1;
         T.res_rows = rows_total;
-        T.SA = (int)std::min<long long>(6, (kSmemBudget - fixed - (long long)rows_total * 128) / T.a_bytes);
+        T.SA = (int)std::min<long long>(4, (kSmemBudget - fixed - (long long)rows_total * 128) / T.a_stride);
         T.SB = 1;
     } else {
-        // input slots first (most that still leave >= 3 weight slots), else 2 + 2
         int best_sa = 0, best_sb = 0;
-        for (int sa = 6; sa >= 2 && !best_sa; --sa) {
-            const long long rest = kSmemBudget - fixed - (long long)sa * T.a_bytes;
+        for (int sa = 4; sa >= 2 && !best_sa; --sa) {
+            const long long rest = kSmemBudget - fixed - (long long)sa * T.a_stride;
             const long long sb = rest / T.b_slot_bytes;
-            if (sb >= 3) {
+            if (sb >= 4 || (sa == 2 && sb >= 2)) {
                 best_sa = sa;
-                best_sb = (int)std::min<long long>(sb, 8);
+                best_sb = (int)std::min<long long>(sb, 12);
             }
-        }
-        if (!best_sa && 2LL * T.a_bytes + 2LL * T.b_slot_bytes + fixed <= kSmemBudget) {
-            best_sa = 2;
-            best_sb = 2;
         }
         if (best_sa == 0) return false;
         T.SA = best_sa;
         T.SB = best_sb;
     }
     return smem_bytes(T) <= (size_t)kSmemBudget;
+}
+
+// Load-path bytes per MMA cycle of a built table set (lower is better).
+double load_rate(const HaloTables &T) {
+    long long cols = 0;
+    for (int i = 0; i < T.n_items; ++i) cols += T.item[i].n;
+    const double mma_clk = (double)T.Mt * cols * 2.0 / T.n_groups;   // per unit and channel block
+    const double a = T.a_bytes;
+    const double b = T.resident ? 0.0 : (double)T.total_rows * 128 / T.KB / T.n_groups;
+    return (a + b) / mma_clk;
+}
+
+// Pick the policy: double-buffered TMEM (Mt x group <= 256 columns) with the
+// lowest load bytes per MMA cycle; single-buffered Mt = 2 as the last resort.
+bool choose_tables(const Plan &p, HaloTables &T) {
+    HaloTables *cand = new HaloTables();
+    bool found = false;
+    double best = 1e30;
+    const int opts[3][2] = {{2, 128}, {1, 256}, {2, 256}};
+    for (int o = 0; o < 3; ++o) {
+        *cand = HaloTables();
+        if (!build_tables(p, *cand, opts[o][0], opts[o][1])) continue;
+        double r = load_rate(*cand);
+        if (cand->nbuf == 1) r *= 1.5;   // the epilogue is not hidden
+        if (r < best) {
+            best = r;
+            T = *cand;
+            found = true;
+        }
+    }
+    delete cand;
+    return found;
 }
 
 }  // namespace
@@ -627,9 +721,8 @@ bool dense_tc_supports(const Plan &p) {
         for (int r = 0; r < p.s[a]; ++r)
             for (const Tap &t : p.taps[a][r])
                 if (t.e < -30000 || t.e > 30000) return false;
-    if (ceil_div(p.out[2], p.s[2]) < 8) return false;   // narrow rows: the per-tap kernel
     HaloTables *T = new HaloTables();
-    const bool ok = build_tables(p, *T, 2, false);
+    const bool ok = choose_tables(p, *T);
     delete T;
     return ok;
 }
@@ -637,14 +730,7 @@ bool dense_tc_supports(const Plan &p) {
 void dense_tc_setup(Plan &p) {
     p.aux.assign((sizeof(HaloTables) + 7) / 8, 0);
     HaloTables &T = *reinterpret_cast<HaloTables *>(p.aux.data());
-    // Mt = 2 (weights feed two pixel tiles) unless the weights are resident
-    // and a single M-tile double-buffers TMEM.
-    build_tables(p, T, 2, false);
-    if (T.resident && T.Mt > 1) {
-        HaloTables *T1 = new HaloTables();
-        if (build_tables(p, *T1, 1, false) && T1->resident) T = *T1;
-        delete T1;
-    }
+    choose_tables(p, T);
     p.launches = 1 + (p.layout == CT_NCHW ? 1 : 0) + (T.dead ? 1 : 0);
 }
 
@@ -683,7 +769,7 @@ ct_status dense_tc_run(const Plan &p, const void *x, const void *wp, const void 
         const cuuint64_t c2 = (cuuint64_t)p.C * 2;
         const cuuint64_t strides[4] = {c2, c2 * p.in[2], c2 * p.in[2] * p.in[1],
                                        c2 * p.in[2] * p.in[1] * p.in[0]};
-        const cuuint32_t box[5] = {64, (cuuint32_t)T.BX, (cuuint32_t)T.BYh, 1, 1};
+        const cuuint32_t box[5] = {64, (cuuint32_t)T.HX, (cuuint32_t)T.HYb, (cuuint32_t)T.HZb, 1};
         const cuuint32_t es[5] = {1, 1, 1, 1, 1};
         if (enc(&tmA, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 5, const_cast<void *>(xa), dims, strides, box, es,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
