@@ -157,3 +157,35 @@ def test_dense_tc_dead_phases_and_degenerate():
         full_parity(dict(x_shape=[2, 136, 23, 70], w_shape=[136, 96, 4, 4], strides=[2, 2],
                          pads=[1, 1, 1, 1], bias=True), torch.float16, 44, layout,
                     algo="dense_tc", expect_kernel="dense_tc")
+
+
+def test_grouped_random_sweep():
+    """fp16 grouped channels-first shapes on the mma.sync grouped phase kernel:
+    ranks 1-2, 16-64 channels per group, strides/dilations up to 3, pads,
+    output_padding, phases without taps (bias only)."""
+    rng = np.random.default_rng(500)
+    for i in range(40):
+        case = random_case(rng, max_rank=2, groups=(2, 4, 8), max_cg=1, max_mg=1,
+                           lim_in={1: 60, 2: 14}, lim_k={1: 5, 2: 4}, strides=(1, 4),
+                           dils=(1, 4))
+        g = case["group"]
+        cg = int(rng.choice([16, 32, 48, 64]))
+        mg = int(rng.choice([8, 16, 24, 40, 64]))
+        case["x_shape"][1] = cg * g
+        case["w_shape"][0] = cg * g
+        case["w_shape"][1] = mg
+        full_parity(case, torch.float16, 9000 + i, "nchw", algo="grouped", expect_kernel="grouped")
+
+
+def test_grouped_bias_only_phases_exact():
+    # the grouped workload's geometry (stride 2, dilation 2, SAME_UPPER) at a
+    # smaller size: 3/4 of the outputs are exactly the bias
+    case = dict(x_shape=[2, 64, 13, 11], w_shape=[64, 16, 3, 3], strides=[2, 2], dilations=[2, 2],
+                auto_pad="SAME_UPPER", group=4, bias=True)
+    x, w, b = draw_case(case, torch.float16, 61)
+    op, y = gpu_run(case, x, w, b, "nchw", "grouped")
+    assert op.kernel == "grouped"
+    bb = b.cuda().view(1, -1, 1, 1)
+    assert torch.equal(y[:, :, 0::2, :], bb.expand_as(y[:, :, 0::2, :]))
+    assert torch.equal(y[:, :, :, 0::2], bb.expand_as(y[:, :, :, 0::2]))
+    full_parity(case, torch.float16, 61, "nchw", algo="grouped", expect_kernel="grouped")

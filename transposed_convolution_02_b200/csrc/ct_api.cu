@@ -239,7 +239,10 @@ ct_status ct_plan(const ct_desc *desc, ct_plan_t **out) {
             p->packed_bytes = dense_pertap_packed_bytes(*p);
             p->ws_bytes = dense_pertap_ws_bytes(*p);
             break;
-        case CT_ALGO_GROUPED: p->packed_bytes = grouped_packed_bytes(*p); break;
+        case CT_ALGO_GROUPED:
+            grouped_plan(*p);
+            p->packed_bytes = grouped_packed_bytes(*p);
+            break;
         case CT_ALGO_FP32_GEMM: p->packed_bytes = fp32_gemm_packed_bytes(*p); break;
         default: p->packed_bytes = generic_packed_bytes(*p); break;
     }

@@ -85,6 +85,7 @@ ct_status fp32_gemm_run(const Plan &p, const void *x, const void *wp, const void
                         cudaStream_t st);
 
 bool grouped_supports(const Plan &p);
+void grouped_plan(Plan &p);
 size_t grouped_packed_bytes(const Plan &p);
 ct_status grouped_prepack(const Plan &p, const void *w, void *wp, cudaStream_t st);
 ct_status grouped_run(const Plan &p, const void *x, const void *wp, const void *bias, void *y,
