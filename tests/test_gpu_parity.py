@@ -189,3 +189,21 @@ def test_grouped_bias_only_phases_exact():
     assert torch.equal(y[:, :, 0::2, :], bb.expand_as(y[:, :, 0::2, :]))
     assert torch.equal(y[:, :, :, 0::2], bb.expand_as(y[:, :, :, 0::2]))
     full_parity(case, torch.float16, 61, "nchw", algo="grouped", expect_kernel="grouped")
+
+
+@pytest.mark.parametrize("layout", ["nchw", "nhwc"])
+def test_fp32_gemm_random_sweep(layout):
+    """fp32 group-1 shapes on the register-tiled FFMA phase GEMM: ranks 1-3,
+    strides/dilations up to 3-4, pads, output_padding, C not a multiple of 8,
+    M not a multiple of 128, phases without taps."""
+    rng = np.random.default_rng(600 + (layout == "nhwc"))
+    for i in range(40):
+        case = random_case(rng, groups=(1,), max_cg=1, max_mg=1,
+                           lim_in={1: 300, 2: 24, 3: 8}, lim_k={1: 9, 2: 5, 3: 3})
+        c = int(rng.choice([1, 3, 8, 20, 64, 72]))
+        m = int(rng.choice([1, 5, 33, 128, 130, 200]))
+        case["x_shape"][1] = c
+        case["w_shape"][0] = c
+        case["w_shape"][1] = m
+        full_parity(case, torch.float32, 11000 + i, layout, algo="fp32_gemm",
+                    expect_kernel="fp32_gemm")

@@ -141,6 +141,9 @@ void choose(Plan *p) {
     const int want = p->desc.algo;
     p->algo = CT_ALGO_GENERIC;
     if (want == CT_ALGO_GENERIC) return;
+    // tiny problems: one gather launch beats any tiled kernel's set-up
+    const double flop = 2.0 * p->N * p->C * p->Mg * numel_in(*p) * numel_k(*p);
+    if (want == CT_ALGO_AUTO && flop < 1e7) return;
     if ((want == CT_ALGO_AUTO || want == CT_ALGO_DENSE_TC) && dense_tc_supports(*p)) {
         p->algo = CT_ALGO_DENSE_TC;
     } else if ((want == CT_ALGO_AUTO || want == CT_ALGO_DENSE_TC || want == CT_ALGO_DENSE_TC_PERTAP) &&
@@ -243,7 +246,10 @@ ct_status ct_plan(const ct_desc *desc, ct_plan_t **out) {
             grouped_plan(*p);
             p->packed_bytes = grouped_packed_bytes(*p);
             break;
-        case CT_ALGO_FP32_GEMM: p->packed_bytes = fp32_gemm_packed_bytes(*p); break;
+        case CT_ALGO_FP32_GEMM:
+            fp32_gemm_plan(*p);
+            p->packed_bytes = fp32_gemm_packed_bytes(*p);
+            break;
         default: p->packed_bytes = generic_packed_bytes(*p); break;
     }
     *out = reinterpret_cast<ct_plan_t *>(p);

@@ -79,6 +79,7 @@ ct_status dense_tc_run(const Plan &p, const void *x, const void *wp, const void 
                        void *ws, cudaStream_t st);
 
 bool fp32_gemm_supports(const Plan &p);
+void fp32_gemm_plan(Plan &p);
 size_t fp32_gemm_packed_bytes(const Plan &p);
 ct_status fp32_gemm_prepack(const Plan &p, const void *w, void *wp, cudaStream_t st);
 ct_status fp32_gemm_run(const Plan &p, const void *x, const void *wp, const void *bias, void *y,
