@@ -21,7 +21,7 @@
 //    TMEM accumulators run as one MMA with a wider N.
 //  * A unit covers Mt tiles of 128 positions, so each weight tile feeds Mt
 //    MMAs; weights stay resident in shared memory when they all fit.
-// Warps: 0 loads input tiles, 1 issues MMAs, 2 loads weights, 4-7 drain TMEM
+// Warps: 0 loads input tiles, 1 issues MMAs, 2-3 load weights, 4-7 drain TMEM
 // (bias from shared memory, fp16 rounding, paired x phases stored as half2).
 #include <cuda.h>
 
@@ -197,7 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *sB = sA + (size_t)SA * a_stride;       // ring slots, or the resident weights
     const size_t b_region = resident ? (size_t)res_rows * 128 : (size_t)SB * b_slot;
     float *bias_s = reinterpret_cast<float *>(sB + b_region);
-    SItem *items_s = reinterpret_cast<SItem *>(bias_s + Np);
+    SItem *items_s = reinterpret_cast<SItem *>(bias_s + ((Np + 31) & ~31));   // bias padded to 32
     SGroup *groups_s = reinterpret_cast<SGroup *>(items_s + n_items);
     int16_t *phr_s = reinterpret_cast<int16_t *>(groups_s + n_groups);
     uint64_t *bars = reinterpret_cast<uint64_t *>(((uintptr_t)(phr_s + 3 * n_phases) + 7) & ~(uintptr_t)7);
@@ -253,7 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         groups_s[g] = gr;
     }
     for (int i = threadIdx.x; i < 3 * n_phases; i += kThreads) phr_s[i] = T.phase_r[i / 3][i % 3];
-    for (int m = threadIdx.x; m < Np; m += kThreads)
+    for (int m = threadIdx.x; m < ((Np + 31) & ~31); m += kThreads)
         bias_s[m] = (T.has_bias && m < M) ? __half2float(bias[m]) : 0.f;
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_slot), 512);
@@ -286,12 +286,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const int first = ia > SA ? ia - SA : 0;
         for (int j = first; j < ia; ++j) mbar_wait(fullA + 8 * (j % SA), (j / SA) & 1, err, 2);
-    } else if (warp == 2 && lane == 0) {
-        // ---------------- weight tiles ----------------
+    } else if ((warp == 2 || warp == 3) && lane == 0) {
+        // ---------------- weight tiles: two issuing warps, alternate ring items ----------------
+        const int me = warp - 2;
         if (resident) {
-            mbar_arrive_expect_tx(bres, (uint32_t)res_rows * 128);
-            for (int r = 0; r < res_rows; r += BR) tma_load_2d(smem_u32(sB + (size_t)r * 128), &tmB, bres, 0, r);
-            mbar_wait(bres, 0, err, 3);
+            if (me == 0) {
+                mbar_arrive_expect_tx(bres, (uint32_t)res_rows * 128);
+                for (int r = 0; r < res_rows; r += BR) tma_load_2d(smem_u32(sB + (size_t)r * 128), &tmB, bres, 0, r);
+                mbar_wait(bres, 0, err, 3);
+            }
         } else {
             int ib = 0;
             bool ok = true;
@@ -301,6 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int kb = 0; kb < KB && ok; ++kb) {
                     const int rowbase = gr.brow + kb * gr.rows_kb;
                     for (int it = gr.item0; it < gr.item0 + gr.nitem; ++it, ++ib) {
+                        if ((ib & 1) != me) continue;
                         const int s = ib % SB;
                         if (ib >= SB && !mbar_wait(emptyB + 8 * s, ((ib / SB) - 1) & 1, err, 4)) {
                             ok = false;
@@ -314,8 +318,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
+            // this warp's copies in flight must land before the CTA exits
             const int first = ib > SB ? ib - SB : 0;
-            for (int j = first; j < ib; ++j) mbar_wait(fullB + 8 * (j % SB), (j / SB) & 1, err, 5);
+            for (int j = first; j < ib; ++j)
+                if ((j & 1) == me) mbar_wait(fullB + 8 * (j % SB), (j / SB) & 1, err, 5);
         }
     } else if (warp == 1 && lane == 0) {
         // ---------------- MMA issue ----------------
@@ -434,20 +440,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                         __half *dst = base + (long long)m0 * cstride;
                         if (!nhwc && pair) {
                             // both x phases of a channel are adjacent: one half2 per channel
+                            float bb[32];
+#pragma unroll
+                            for (int j = 0; j < 8; ++j)
+                                *reinterpret_cast<float4 *>(&bb[4 * j]) =
+                                    *reinterpret_cast<const float4 *>(&bias_s[m0 + 4 * j]);
 #pragma unroll
                             for (int j = 0; j < 16; ++j)
                                 if (j < mc0)
                                     *reinterpret_cast<__half2 *>(dst + j * plane) =
-                                        __floats2half2_rn(__uint_as_float(v0[j]) + bias_s[m0 + j],
-                                                          __uint_as_float(w0[j]) + bias_s[m0 + j]);
+                                        __floats2half2_rn(__uint_as_float(v0[j]) + bb[j],
+                                                          __uint_as_float(w0[j]) + bb[j]);
                             if (two) {
                                 __half *d1 = dst + 16 * plane;
 #pragma unroll
                                 for (int j = 0; j < 16; ++j)
                                     if (j < mc1)
                                         *reinterpret_cast<__half2 *>(d1 + j * plane) =
-                                            __floats2half2_rn(__uint_as_float(v1[j]) + bias_s[m0 + 16 + j],
-                                                              __uint_as_float(w1[j]) + bias_s[m0 + 16 + j]);
+                                            __floats2half2_rn(__uint_as_float(v1[j]) + bb[16 + j],
+                                                              __uint_as_float(w1[j]) + bb[16 + j]);
                             }
                         } else {
                             store_chunk16(dst, cstride, v0, bias_s + m0, mc0);
@@ -477,7 +488,7 @@ size_t smem_bytes(const HaloTables &T) {
     const size_t b_region = T.resident ? (size_t)T.res_rows * 128 : (size_t)T.SB * T.b_slot_bytes;
     const size_t tables = (size_t)T.n_items * sizeof(SItem) + (size_t)T.n_groups * sizeof(SGroup) +
                           (size_t)T.n_phases * 6 + 8;
-    return 1024 + (size_t)T.SA * T.a_stride + b_region + (size_t)T.Np * 4 + tables +
+    return 1024 + (size_t)T.SA * T.a_stride + b_region + (size_t)((T.Np + 31) & ~31) * 4 + tables +
            (size_t)(2 * T.SA + 2 * T.SB + 6) * 8 + 16;
 }
 
@@ -652,7 +663,7 @@ bool build_tables(const Plan &p, HaloTables &T, int Mt, int gmax_cols) {
     for (int i = 0; i < ni; ++i) nmax = std::max(nmax, (int)T.item[i].n);
     T.b_slot_bytes = nmax * 128;
     // shared memory: resident weights if they fit next to two input slots
-    const int fixed = 1024 + T.Np * 4 + 64 * 8 + 64 + ni * (int)sizeof(SItem) + ng * (int)sizeof(SGroup) +
+    const int fixed = 1024 + ((T.Np + 31) & ~31) * 4 + 64 * 8 + 64 + ni * (int)sizeof(SItem) + ng * (int)sizeof(SGroup) +
                       np * 6 + 8;
     T.resident = 0;
     T.res_rows = 0;
@@ -678,36 +689,18 @@ bool build_tables(const Plan &p, HaloTables &T, int Mt, int gmax_cols) {
     return smem_bytes(T) <= (size_t)kSmemBudget;
 }
 
-// Load-path bytes per MMA cycle of a built table set (lower is better).
-double load_rate(const HaloTables &T) {
-    long long cols = 0;
-    for (int i = 0; i < T.n_items; ++i) cols += T.item[i].n;
-    const double mma_clk = (double)T.Mt * cols * 2.0 / T.n_groups;   // per unit and channel block
-    const double a = T.a_bytes;
-    const double b = T.resident ? 0.0 : (double)T.total_rows * 128 / T.KB / T.n_groups;
-    return (a + b) / mma_clk;
-}
-
-// Pick the policy: double-buffered TMEM (Mt x group <= 256 columns) with the
-// lowest load bytes per MMA cycle; single-buffered Mt = 2 as the last resort.
+// Pick the layout: Mt x group of accumulator columns.  Measured on a B200
+// (2-D fp16 decoder and 3-D fp16 upsample workloads), two M-tiles with both x
+// phases of a pair in one group (TMEM single-buffered, whole-line half2
+// stores, half the weight traffic per pixel) is fastest, then one M-tile with
+// paired phases (double-buffered), then two M-tiles of lone phases.
 bool choose_tables(const Plan &p, HaloTables &T) {
-    HaloTables *cand = new HaloTables();
-    bool found = false;
-    double best = 1e30;
-    const int opts[3][2] = {{2, 128}, {1, 256}, {2, 256}};
+    const int opts[3][2] = {{2, 256}, {1, 256}, {2, 128}};
     for (int o = 0; o < 3; ++o) {
-        *cand = HaloTables();
-        if (!build_tables(p, *cand, opts[o][0], opts[o][1])) continue;
-        double r = load_rate(*cand);
-        if (cand->nbuf == 1) r *= 1.5;   // the epilogue is not hidden
-        if (r < best) {
-            best = r;
-            T = *cand;
-            found = true;
-        }
+        T = HaloTables();
+        if (build_tables(p, T, opts[o][0], opts[o][1])) return true;
     }
-    delete cand;
-    return found;
+    return false;
 }
 
 }  // namespace
