@@ -191,6 +191,33 @@ def test_grouped_bias_only_phases_exact():
     full_parity(case, torch.float16, 61, "nchw", algo="grouped", expect_kernel="grouped")
 
 
+@pytest.mark.parametrize("case", [
+    # one stride phase with taps in each axis (stride 2, dilation 2, kernel 3):
+    # 16-byte stores (out_x % 8 == 0), a ragged segment and row-block tail
+    dict(x_shape=[2, 32, 13, 12], w_shape=[32, 16, 3, 3], strides=[2, 2], dilations=[2, 2],
+         auto_pad="SAME_UPPER", group=2, bias=True),
+    # 8-byte stores (out_x % 8 == 4), half an output-channel tile (M/group = 8)
+    dict(x_shape=[3, 64, 7, 10], w_shape=[64, 8, 3, 3], strides=[2, 2], dilations=[2, 2],
+         auto_pad="SAME_UPPER", group=4, bias=True),
+    # the even column phase carries the taps (SAME_LOWER), no bias
+    dict(x_shape=[2, 32, 9, 16], w_shape=[32, 16, 3, 3], strides=[2, 2], dilations=[2, 2],
+         auto_pad="SAME_LOWER", group=2, bias=False),
+    # rank 1
+    dict(x_shape=[2, 48, 40], w_shape=[48, 16, 3], strides=[2], dilations=[2],
+         auto_pad="SAME_UPPER", group=3, bias=True),
+    # one tap (kernel 1, output_padding 1) and two k-steps per tap (32 channels per group)
+    dict(x_shape=[2, 64, 8, 8], w_shape=[64, 16, 1, 1], strides=[2, 2], output_padding=[1, 1],
+         group=2, bias=True),
+    # four taps (kernel 2, dilation 2, output_padding 1 so that out_x % 4 == 0)
+    dict(x_shape=[2, 32, 11, 11], w_shape=[32, 8, 2, 2], strides=[2, 2], dilations=[2, 2],
+         output_padding=[1, 1], group=2, bias=True),
+])
+def test_grouped_one_phase_path(case):
+    """Grouped shapes whose outputs get taps in one stride phase only (the
+    path that keeps the weights in registers and stores (bias, value) pairs)."""
+    full_parity(case, torch.float16, 70, "nchw", algo="grouped", expect_kernel="grouped")
+
+
 @pytest.mark.parametrize("layout", ["nchw", "nhwc"])
 def test_fp32_gemm_random_sweep(layout):
     """fp32 group-1 shapes on the register-tiled FFMA phase GEMM: ranks 1-3,
