@@ -222,6 +222,28 @@ def time_device(wl, device, steps, warmup, l2_bytes, dist_max=None, sampler=None
     return ms, info
 
 
+def make_dist_max(dist, device=None):
+    """Collective helpers over the default process group: a barrier, and the
+    maximum of one float over all ranks (every rank takes the same steps)."""
+    def dist_max(what, value=None):
+        if what == "barrier":
+            dist.barrier()
+            return None
+        t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+    return dist_max
+
+
+def aggregate(flop_per_replica, ms_local, steps, world, dist_max=None):
+    """Whole-job rate of `world` independent replicas: every rank processed
+    one replica per step, the job took the slowest rank's time.  Returns
+    (ms for `steps` steps, TFLOP/s over all ranks)."""
+    ms = dist_max("max", ms_local) if dist_max is not None else ms_local
+    sec_per_step = ms / 1e3 / steps
+    return ms, flop_per_replica * max(world, 1) / sec_per_step / 1e12
+
+
 class _Null:
     def __enter__(self):
         return self
@@ -377,14 +399,7 @@ def main():
         import torch.distributed as dist
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-
-        def dist_max(what, value=None):
-            if what == "barrier":
-                dist.barrier()
-                return None
-            t = torch.tensor([value], dtype=torch.float64, device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            return float(t.item())
+        dist_max = make_dist_max(dist, device=torch.device("cuda", local))
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     props = torch.cuda.get_device_properties(device)
@@ -393,10 +408,8 @@ def main():
 
     sampler = ClockSampler(local)
     ms, info = time_device(wl, device, args.steps, args.warmup, l2, dist_max, sampler)
-    if dist_max is not None:
-        ms = dist_max("max", ms)
+    ms, value = aggregate(flop, ms, args.steps, world, dist_max)
     sec_per_step = ms / 1e3 / args.steps
-    value = flop * max(world, 1) / sec_per_step / 1e12
     roof = roofline_for(wl, sec_per_step, peaks, props.multi_processor_count)
     roof["peak_source"] = peaks["source"] + " (burst)"
     roof["traffic"] = traffic_for(info["kernel"])
@@ -405,9 +418,7 @@ def main():
 
     e2e_steps = max(3, min(args.steps, 50))
     ems, hb, db = time_e2e(wl, device, e2e_steps, 3)
-    if dist_max is not None:
-        ems = dist_max("max", ems)
-    e2e_value = flop * max(world, 1) / (ems / 1e3 / e2e_steps) / 1e12
+    ems, e2e_value = aggregate(flop, ems, e2e_steps, world, dist_max)
 
     others = {}
     if not args.no_others:
