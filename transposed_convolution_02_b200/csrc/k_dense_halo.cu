@@ -327,7 +327,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---------------- MMA issue ----------------
         bool ok = true;
         if (resident) ok = mbar_wait(bres, 0, err, 6);
-        int ia = 0, ib = 0, local = 0;
+        int ia = 0, local = 0;
+        uint32_t sb_slot = 0, sb_phase = 0;   // weight ring position of the next item
         for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++local) {
             const Unit U = decode_unit(G, u);
             const SGroup gr = groups_s[U.g];
@@ -362,23 +363,31 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (Mt > 1) issue4(d + mstep, ad + 1024, bd, idesc, acc0);   // +128 rows
                     }
                 } else {
+                    // Shared-memory reads of this thread wait behind the MMAs'
+                    // operand reads, so the next item's entry is fetched before
+                    // the current item's MMAs are issued, and the ring slot and
+                    // phase advance by counters instead of divisions.
+                    SItem In = items_s[i0];
                     for (int it = i0; it < i1; ++it) {
-                        const SItem I = items_s[it];
-                        const int sb = ib % SB;
-                        if (!mbar_wait(fullB + 8 * sb, (ib / SB) & 1, err, 9)) {
+                        const SItem I = In;
+                        if (it + 1 < i1) In = items_s[it + 1];
+                        if (!mbar_wait(fullB + 8 * sb_slot, sb_phase, err, 9)) {
                             ok = false;
                             break;
                         }
                         tc_fence_after();
-                        const uint64_t bd = desc_kmajor_sw128(smem_u32(sB + (size_t)sb * b_slot));
+                        const uint64_t bd = desc_kmajor_sw128(smem_u32(sB) + sb_slot * (uint32_t)b_slot);
                         const uint64_t ad = desc_kmajor_sw128(a_addr + (uint32_t)I.shift * 128);
                         const uint32_t idesc = idesc_f16_f32(128, I.n);
                         const uint32_t d = dbase + I.tcol;
                         const uint32_t acc0 = (kb == 0 && I.first) ? 0u : 1u;
                         issue4(d, ad, bd, idesc, acc0);
                         if (Mt > 1) issue4(d + mstep, ad + 1024, bd, idesc, acc0);   // +128 rows
-                        mma_commit(emptyB + 8 * sb);
-                        ++ib;
+                        mma_commit(emptyB + 8 * sb_slot);
+                        if (++sb_slot == (uint32_t)SB) {
+                            sb_slot = 0;
+                            sb_phase ^= 1u;
+                        }
                     }
                 }
                 mma_commit(emptyA + 8 * sa);
