@@ -159,6 +159,17 @@ def test_dense_tc_dead_phases_and_degenerate():
                     algo="dense_tc", expect_kernel="dense_tc")
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.float16])
+def test_generic_untabled_stride(dtype):
+    """Stride 80 (more phases than the phase tables hold): the generic
+    kernel's 64-bit form, which tests every tap."""
+    full_parity(dict(x_shape=[2, 4, 5], w_shape=[4, 3, 3], strides=[80], bias=True), dtype, 80,
+                "nchw", algo="generic", expect_kernel="generic")
+    full_parity(dict(x_shape=[1, 6, 3, 2], w_shape=[6, 2, 2, 3], strides=[70, 3], dilations=[2, 1],
+                     pads=[3, 1, 0, 2], group=2, bias=True), dtype, 81, "nhwc", algo="generic",
+                expect_kernel="generic")
+
+
 def test_grouped_random_sweep():
     """fp16 grouped channels-first shapes on the mma.sync grouped phase kernel:
     ranks 1-2, 16-64 channels per group, strides/dilations up to 3, pads,

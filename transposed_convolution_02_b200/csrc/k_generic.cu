@@ -3,10 +3,19 @@
 // dilation, padding, group, layout and both dtypes; the specialised kernels
 // take the shapes that matter for speed.
 //
+// Two forms: when every index fits in 32 bits and the strides have phase
+// tables, a thread splits each output coordinate o into o = s*J + r (r the
+// stride phase) once and walks only the taps of phase r, reading input
+// J + e (e the tap's offset); every division is a precomputed multiply-shift.
+// Otherwise a 64-bit form tests every tap.
+//
 // For output position o on an axis with stride s, dilation d and begin pad pb,
 // tap k contributes iff (o + pb - k*d) is a non-negative multiple of s, and
 // it reads input position i = (o + pb - k*d) / s (ai.onnx.ConvTranspose
 // README, "Description": the scatter o = i*s - pb + k*d read backwards).
+#include <algorithm>
+
+#include "ct_divmagic.h"
 #include "ct_internal.h"
 
 namespace ct {
@@ -96,6 +105,126 @@ __global__ void __launch_bounds__(256) generic_kernel(GenericArgs a, const T *__
     }
 }
 
+constexpr int kG32MaxS = 64;      // phases per axis
+constexpr int kG32MaxTaps = 64;   // taps per axis
+
+struct Generic32Args {
+    int32_t C, M, Cg, Mg, in_sz, k_sz, total, nhwc, has_bias;
+    int32_t in[3], out[3], s[3], kst[3];     // kpos = k0*kst[0] + k1*kst[1] + k2*kst[2]
+    DivMagic d_out[3], d_M, d_Mg, d_s[3];
+    uint8_t ph_off[3][kG32MaxS], ph_cnt[3][kG32MaxS];   // taps of phase r of axis a
+    int16_t tap_e[3][kG32MaxTaps], tap_k[3][kG32MaxTaps];
+};
+
+template <typename T>
+__global__ void __launch_bounds__(256, 4) generic32_kernel(const __grid_constant__ Generic32Args a,
+                                                        const T *__restrict__ x, const T *__restrict__ w,
+                                                        const T *__restrict__ bias, T *__restrict__ y) {
+    for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < a.total; idx += gridDim.x * blockDim.x) {
+        // idx -> (n, m, o0, o1, o2) in the layout's order
+        int rem = idx, m = 0;
+        if (a.nhwc) {
+            const int q = divq(rem, a.d_M);
+            m = rem - q * a.M;
+            rem = q;
+        }
+        int q = divq(rem, a.d_out[2]);
+        const int o2 = rem - q * a.out[2];
+        rem = q;
+        q = divq(rem, a.d_out[1]);
+        const int o1 = rem - q * a.out[1];
+        rem = q;
+        q = divq(rem, a.d_out[0]);
+        const int o0 = rem - q * a.out[0];
+        rem = q;
+        if (!a.nhwc) {
+            q = divq(rem, a.d_M);
+            m = rem - q * a.M;
+            rem = q;
+        }
+        const int n = rem;
+        const int g = divq(m, a.d_Mg), ml = m - g * a.Mg;
+        // o = s*J + r on every axis
+        const int J0 = divq(o0, a.d_s[0]), r0 = o0 - J0 * a.s[0];
+        const int J1 = divq(o1, a.d_s[1]), r1 = o1 - J1 * a.s[1];
+        const int J2 = divq(o2, a.d_s[2]), r2 = o2 - J2 * a.s[2];
+        float acc = 0.f;
+        const int q0b = a.ph_off[0][r0], q0e = q0b + a.ph_cnt[0][r0];
+        const int q1b = a.ph_off[1][r1], q1e = q1b + a.ph_cnt[1][r1];
+        const int q2b = a.ph_off[2][r2], q2e = q2b + a.ph_cnt[2][r2];
+        for (int q0 = q0b; q0 < q0e; ++q0) {
+            const int i0 = J0 + a.tap_e[0][q0];
+            if ((unsigned)i0 >= (unsigned)a.in[0]) continue;
+            for (int q1 = q1b; q1 < q1e; ++q1) {
+                const int i1 = J1 + a.tap_e[1][q1];
+                if ((unsigned)i1 >= (unsigned)a.in[1]) continue;
+                for (int q2 = q2b; q2 < q2e; ++q2) {
+                    const int i2 = J2 + a.tap_e[2][q2];
+                    if ((unsigned)i2 >= (unsigned)a.in[2]) continue;
+                    const int ipos = (i0 * a.in[1] + i1) * a.in[2] + i2;
+                    const int kpos = a.tap_k[0][q0] * a.kst[0] + a.tap_k[1][q1] * a.kst[1] + a.tap_k[2][q2] * a.kst[2];
+                    const int c0 = g * a.Cg;
+                    if (a.nhwc) {
+                        const T *xp = x + (n * a.in_sz + ipos) * a.C + c0;
+                        const T *wp = w + (c0 * a.k_sz + kpos) * a.Mg + ml;
+                        for (int cl = 0; cl < a.Cg; ++cl)
+                            acc = fmaf(to_f(xp[cl]), to_f(wp[cl * a.k_sz * a.Mg]), acc);
+                    } else {
+                        const T *xp = x + (n * a.C + c0) * a.in_sz + ipos;
+                        const T *wp = w + (c0 * a.Mg + ml) * a.k_sz + kpos;
+                        for (int cl = 0; cl < a.Cg; ++cl)
+                            acc = fmaf(to_f(xp[cl * a.in_sz]), to_f(wp[cl * a.Mg * a.k_sz]), acc);
+                    }
+                }
+            }
+        }
+        if (a.has_bias) acc += to_f(bias[m]);
+        y[idx] = from_f<T>(acc);
+    }
+}
+
+// The 32-bit form's arguments; false when an index or table would not fit.
+bool generic32_setup(const Plan &p, Generic32Args &a) {
+    const int64_t lim = (int64_t)1 << 31;
+    const int64_t total = p.N * p.M * numel_out(p);
+    if (!p.tabled || total >= lim || p.N * p.C * numel_in(p) >= lim || p.C * p.Mg * numel_k(p) >= lim) return false;
+    a = Generic32Args();
+    a.C = (int32_t)p.C;
+    a.M = (int32_t)p.M;
+    a.Cg = (int32_t)p.Cg;
+    a.Mg = (int32_t)p.Mg;
+    a.in_sz = (int32_t)numel_in(p);
+    a.k_sz = (int32_t)numel_k(p);
+    a.total = (int32_t)total;
+    a.nhwc = p.layout == CT_NHWC;
+    a.has_bias = p.has_bias;
+    a.kst[2] = 1;
+    a.kst[1] = (int32_t)p.k[2];
+    a.kst[0] = (int32_t)(p.k[1] * p.k[2]);
+    for (int ax = 0; ax < 3; ++ax) {
+        if (p.s[ax] > kG32MaxS || p.k[ax] > kG32MaxTaps || p.out[ax] < 1) return false;
+        a.in[ax] = (int32_t)p.in[ax];
+        a.out[ax] = (int32_t)p.out[ax];
+        a.s[ax] = (int32_t)p.s[ax];
+        a.d_out[ax] = make_magic((uint32_t)p.out[ax]);
+        a.d_s[ax] = make_magic((uint32_t)p.s[ax]);
+        int t = 0;
+        for (int r = 0; r < p.s[ax]; ++r) {
+            a.ph_off[ax][r] = (uint8_t)t;
+            for (const Tap &tp : p.taps[ax][r]) {
+                if (t >= kG32MaxTaps || tp.e < -32768 || tp.e > 32767) return false;
+                a.tap_e[ax][t] = (int16_t)tp.e;
+                a.tap_k[ax][t] = (int16_t)tp.k;
+                ++t;
+            }
+            a.ph_cnt[ax][r] = (uint8_t)(t - a.ph_off[ax][r]);
+        }
+    }
+    a.d_M = make_magic((uint32_t)std::max<int64_t>(1, p.M));
+    a.d_Mg = make_magic((uint32_t)std::max<int64_t>(1, p.Mg));
+    return true;
+}
+
 }  // namespace
 
 bool generic_supports(const Plan &) { return true; }
@@ -129,6 +258,20 @@ ct_status generic_run(const Plan &p, const void *x, const void *wp, const void *
     a.has_bias = p.has_bias;
     if (a.total == 0) return CT_OK;
     const int threads = 256;
+    {
+        Generic32Args b;
+        if (generic32_setup(p, b)) {
+            int64_t blocks32 = ceil_div(b.total, threads);
+            if (blocks32 > 148 * 64) blocks32 = 148 * 64;
+            if (p.dtype == CT_F16)
+                generic32_kernel<__half><<<(unsigned)blocks32, threads, 0, st>>>(
+                    b, (const __half *)x, (const __half *)wp, (const __half *)bias, (__half *)y);
+            else
+                generic32_kernel<float><<<(unsigned)blocks32, threads, 0, st>>>(
+                    b, (const float *)x, (const float *)wp, (const float *)bias, (float *)y);
+            return launch_status();
+        }
+    }
     int64_t blocks = ceil_div(a.total, threads);
     if (blocks > 148 * 64) blocks = 148 * 64;
     if (p.dtype == CT_F16)

@@ -35,6 +35,7 @@
 #include <atomic>
 
 #include "ct_cuda_util.h"
+#include "ct_divmagic.h"
 #include "ct_internal.h"
 #include "sm100.cuh"
 
@@ -55,26 +56,6 @@ constexpr int kGMaxS = 8;
 constexpr int kGMaxPairs = 64;
 constexpr int kGMaxSteps = 320;   // (tap pair, k-step) entries, each phase padded to a multiple of 4
 constexpr int kGSmem = 200 * 1024;
-
-// Division by a run-time invariant d > 0 through a multiply (Granlund and
-// Montgomery, "Division by invariant integers using multiplication", 1994):
-// with l = ceil(log2 d) and m = floor(2^32 (2^l - d) / d) + 1,
-// floor(t / d) = (umulhi(t, m) + t) >> l for every t < 2^31.
-struct DivMagic {
-    uint32_t m;
-    int32_t l;
-};
-
-DivMagic make_magic(uint32_t d) {
-    int l = 0;
-    while ((1ull << l) < d) ++l;
-    const uint64_t m = ((1ull << 32) * ((1ull << l) - d)) / d + 1;
-    return DivMagic{(uint32_t)m, l};
-}
-
-__device__ __forceinline__ int divq(int t, DivMagic d) {
-    return (int)((__umulhi((uint32_t)t, d.m) + (uint32_t)t) >> d.l);
-}
 
 struct GroupedArgs {
     int32_t N, C, M, G, Cg, Mg, KS, MT;     // KS = Cg/16 k-steps, MT = ceil(Mg/16) m-tiles
