@@ -86,21 +86,41 @@ def roofline_for(wl, seconds_per_launch, peaks, sms):
                 frac=a / peaks["hbm_gbs"])
 
 
-def traffic_for(kernel):
-    """DRAM bytes per launch from a committed ncu summary, if the kernel source
-    is unchanged since the capture (else None)."""
+def profile_record(wid, kernel):
+    """The committed ncu record of the workload's dominant kernel (DRAM bytes
+    per launch, its share of one call), if that kernel's source is unchanged
+    since the capture (else None)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
-        rec = json.load(f).get(kernel)
-    if not rec:
+        rec = json.load(f).get(str(wid))
+    if not rec or rec.get("kernel") != kernel:
         return None
     src = os.path.join(ROOT, "transposed_convolution_02_b200", "csrc", rec["source"])
     if not os.path.exists(src):
         return None
     h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    return rec["bytes_per_launch"] if h == rec["sha256_16"] else None
+    return rec if h == rec["sha256_16"] else None
+
+
+def traffic_for(wid, kernel):
+    rec = profile_record(wid, kernel)
+    return rec["bytes_per_launch"] if rec else None
+
+
+def annotate_roofline(roof, wid, kernel, launches):
+    """Scope of the achieved figure: it is measured over whole calls (all of a
+    call's launches); with the dominant kernel's share of a call from the
+    committed launch list, the kernel-only fraction follows."""
+    roof["traffic"] = traffic_for(wid, kernel)
+    roof["kernel"] = kernel
+    roof["scope"] = "whole call (%d launch%s), CUDA events" % (launches, "" if launches == 1 else "es")
+    rec = profile_record(wid, kernel)
+    if rec and launches > 1 and rec.get("share_of_call"):
+        roof["kernel_share_of_call"] = rec["share_of_call"]
+        roof["kernel_frac_est"] = roof["frac"] / rec["share_of_call"]
+    return roof
 
 
 # ---------------------------------------------------------------------------
@@ -412,9 +432,8 @@ def main():
     sec_per_step = ms / 1e3 / args.steps
     roof = roofline_for(wl, sec_per_step, peaks, props.multi_processor_count)
     roof["peak_source"] = peaks["source"] + " (burst)"
-    roof["traffic"] = traffic_for(info["kernel"])
-    roof["kernel"] = info["kernel"]
-    roof["per_launch_us"] = sec_per_step * 1e6 / max(1, info["launches_per_step"])
+    annotate_roofline(roof, args.workload, info["kernel"], info["launches_per_step"])
+    roof["per_call_us"] = sec_per_step * 1e6
 
     e2e_steps = max(3, min(args.steps, 50))
     ems, hb, db = time_e2e(wl, device, e2e_steps, 3)
@@ -433,6 +452,7 @@ def main():
                 oms = dist_max("max", oms)
             osec = oms / 1e3 / osteps
             oroof = roofline_for(owl, osec, peaks, props.multi_processor_count)
+            annotate_roofline(oroof, wid, oinfo["kernel"], oinfo["launches_per_step"])
             others[str(wid)] = {"workload": owl.name, "kernel": oinfo["kernel"],
                                 "us_per_step": osec * 1e6, "tflops": ofl / osec / 1e12,
                                 "roofline": oroof}
