@@ -89,6 +89,16 @@ typedef enum ct_algo {
                                    (the general fallback of CT_ALGO_DENSE_TC) */
 } ct_algo;
 
+/* Activation applied to every output after the bias (ClikaRT::ops::
+ * conv_transpose, parameter `activation`, default Identity).  The page does
+ * not list the Activation members; this library offers identity and ReLU
+ * (max(v, 0)), applied in fp32 before the output is rounded to its dtype.
+ * Any other value is CT_ERR_ATTR. */
+typedef enum ct_activation {
+    CT_ACT_IDENTITY = 0,
+    CT_ACT_RELU = 1
+} ct_activation;
+
 /* One ConvTranspose call.  Every array has 3 slots; only the first `rank`
  * (and 2*rank for pads) are read. */
 typedef struct ct_desc {
@@ -112,7 +122,7 @@ typedef struct ct_desc {
     int64_t kernel_shape[3];
     int64_t output_shape[3];
     int32_t algo;              /* ct_algo */
-    int32_t reserved;
+    int32_t activation;        /* ct_activation */
 } ct_desc;
 
 typedef struct ct_plan_s ct_plan_t;

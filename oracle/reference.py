@@ -80,8 +80,24 @@ def _geometry(x, w, bias, attrs):
     return yshape, res, rank, s, d
 
 
-def conv_transpose_ref(x, w, bias=None, attrs: Attrs = None):
-    """Return (Y, A) in fp64: Y per the scatter definition, A = sum |x*w|."""
+ACTIVATIONS = ("identity", "relu")
+
+
+def apply_activation(y, activation="identity"):
+    """The output activation of ClikaRT::ops::conv_transpose (parameter
+    `activation`, default Identity), applied to the output after the bias.
+    The page names the parameter but not the members of its enum; the two
+    read here are identity and ReLU, max(y, 0)."""
+    if activation == "identity":
+        return y
+    if activation == "relu":
+        return np.maximum(y, 0.0)
+    raise ValueError("unknown activation %r" % (activation,))
+
+
+def conv_transpose_ref(x, w, bias=None, attrs: Attrs = None, activation="identity"):
+    """Return (Y, A) in fp64: Y per the scatter definition (then the
+    activation), A = sum |x*w|."""
     attrs = attrs or Attrs(strides=None)
     yshape, res, rank, s, d = _geometry(x, w, bias, attrs)
     N, C = x.shape[0], x.shape[1]
@@ -107,10 +123,10 @@ def conv_transpose_ref(x, w, bias=None, attrs: Attrs = None):
         a.ctypes.data_as(ctypes.POINTER(ctypes.c_double)))
     if rc != 0:
         raise RuntimeError("oracle rejected the geometry (code %d)" % rc)
-    return y, a
+    return apply_activation(y, activation), a
 
 
-def conv_transpose_points(x, w, bias, attrs: Attrs, points):
+def conv_transpose_points(x, w, bias, attrs: Attrs, points, activation="identity"):
     """Evaluate Y and A at output points (rows of n, m, o_1..o_r)."""
     yshape, res, rank, s, d = _geometry(x, w, bias, attrs)
     N, C = x.shape[0], x.shape[1]
@@ -138,7 +154,7 @@ def conv_transpose_points(x, w, bias, attrs: Attrs, points):
         av.ctypes.data_as(ctypes.POINTER(ctypes.c_double)))
     if rc != 0:
         raise RuntimeError("oracle rejected the points (code %d)" % rc)
-    return yv, av
+    return apply_activation(yv, activation), av
 
 
 def forward_conv_ref(u, wf, strides, dilations, pad_begin, out_spatial, group):

@@ -47,7 +47,8 @@ def gpu_run(case, x, w, b, layout, algo="auto", poison=True):
                           output_padding=case.get("output_padding"),
                           auto_pad=case.get("auto_pad", "NOTSET"), group=case.get("group", 1),
                           kernel_shape=case.get("kernel_shape"),
-                          output_shape=case.get("output_shape"), algo=algo)
+                          output_shape=case.get("output_shape"), algo=algo,
+                          activation=case.get("activation", "identity"))
     y = torch.empty(op.y_shape, dtype=x.dtype, device="cuda")
     if poison:
         y.fill_(float("nan"))
@@ -77,7 +78,8 @@ def full_parity(case, dtype, seed, layout="nchw", algo="auto", expect_kernel=Non
     if expect_kernel is not None:
         assert op.kernel == expect_kernel, (op.kernel, expect_kernel)
     xa, wa, ba = to_oracle(x, w, b, layout)
-    ref, absacc = conv_transpose_ref(xa, wa, ba, attrs_from(case))
+    ref, absacc = conv_transpose_ref(xa, wa, ba, attrs_from(case),
+                                     activation=case.get("activation", "identity"))
     if layout == "nhwc":
         ref = np.moveaxis(ref, 1, -1)
         absacc = np.moveaxis(absacc, 1, -1)
@@ -108,6 +110,7 @@ def sampled_parity(op, y, x, w, b, case, dtype, layout, rng, n_random=1500):
     xa, wa, ba = to_oracle(x, w, b, layout)
     ycf = y if layout == "nchw" else y.movedim(-1, 1)
     pts = sampled_points(list(ycf.shape), rng, n_random)
-    ref, absacc = conv_transpose_points(xa, wa, ba, attrs_from(case), pts)
+    ref, absacc = conv_transpose_points(xa, wa, ba, attrs_from(case), pts,
+                                        activation=case.get("activation", "identity"))
     got = ycf[tuple(torch.from_numpy(pts.T).to(y.device))].double().cpu().numpy()
     return check_close(got, ref, absacc, dtype, "sampled " + str(case))

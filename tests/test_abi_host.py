@@ -131,6 +131,13 @@ def test_error_classes():
     with pytest.raises(ct.CtError) as e:
         ct.ct_output_shape(d)
     assert e.value.status == 3
+    d = _desc_from_case(base)
+    d.activation = 2                                  # only identity (0) and relu (1)
+    with pytest.raises(ct.CtError) as e:
+        ct.ct_output_shape(d)
+    assert e.value.status == 4
+    d.activation = 1
+    ct.ct_output_shape(d)
 
 
 @pytest.mark.parametrize("wid", sorted(WORKLOADS))

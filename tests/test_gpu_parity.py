@@ -159,6 +159,33 @@ def test_dense_tc_dead_phases_and_degenerate():
                     algo="dense_tc", expect_kernel="dense_tc")
 
 
+@pytest.mark.parametrize("algo,dtype,layout,case", [
+    ("generic", torch.float32, "nchw", dict(x_shape=[2, 6, 7], w_shape=[6, 4, 3], strides=[2],
+                                            pads=[1, 0], group=2, bias=True)),
+    ("generic", torch.float16, "nhwc", dict(x_shape=[2, 4, 5, 6], w_shape=[4, 3, 3, 3], strides=[2, 1],
+                                            bias=True)),
+    ("generic", torch.float32, "nchw", dict(x_shape=[1, 3, 4], w_shape=[3, 2, 3], strides=[90], bias=True)),
+    ("dense_tc", torch.float16, "nchw", dict(x_shape=[2, 64, 9, 20], w_shape=[64, 48, 4, 4], strides=[2, 2],
+                                             pads=[1, 1, 1, 1], bias=True)),
+    ("dense_tc", torch.float16, "nchw", dict(x_shape=[2, 32, 5, 6, 12], w_shape=[32, 32, 3, 3, 3],
+                                             strides=[2, 2, 2], dilations=[2, 2, 2], auto_pad="SAME_UPPER",
+                                             bias=True)),
+    ("dense_tc_pertap", torch.float16, "nhwc", dict(x_shape=[2, 32, 6, 5], w_shape=[32, 16, 3, 3],
+                                                    strides=[2, 2], pads=[1, 1, 1, 1], bias=True)),
+    ("fp32_gemm", torch.float32, "nchw", dict(x_shape=[2, 24, 40], w_shape=[24, 40, 4], strides=[4],
+                                              dilations=[2], pads=[1, 2], bias=True)),
+    ("grouped", torch.float16, "nchw", dict(x_shape=[2, 32, 9, 16], w_shape=[32, 16, 3, 3], strides=[2, 2],
+                                            dilations=[2, 2], auto_pad="SAME_UPPER", group=2, bias=True)),
+    ("grouped", torch.float16, "nchw", dict(x_shape=[2, 64, 7, 9], w_shape=[64, 24, 2, 2], strides=[3, 3],
+                                            group=2, bias=True)),
+])
+def test_relu_activation(algo, dtype, layout, case):
+    """The ReLU activation after the bias, in every kernel family and in the
+    bias-only outputs of tap-less phases."""
+    case = dict(case, activation="relu")
+    full_parity(case, dtype, 90, layout, algo=algo, expect_kernel=algo)
+
+
 @pytest.mark.parametrize("dtype", [torch.float32, torch.float16])
 def test_generic_untabled_stride(dtype):
     """Stride 80 (more phases than the phase tables hold): the generic

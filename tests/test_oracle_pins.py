@@ -154,6 +154,32 @@ def test_against_torch_library_sweep():
         np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12, err_msg=str(case))
 
 
+def test_relu_activation_against_torch_library():
+    # ClikaRT::ops::conv_transpose, parameter `activation`: ReLU after the
+    # bias.  Pinned to torch.relu applied to the library special case, and to
+    # the bias-only positions of a stride-2 dilation-2 shape (ReLU of the bias).
+    rng = np.random.default_rng(77)
+    for _ in range(30):
+        case = random_case(rng)
+        attrs = attrs_of(case)
+        x = rng.standard_normal(case["x_shape"])
+        w = rng.standard_normal(case["w_shape"])
+        b = rng.standard_normal(case["w_shape"][1] * case["group"]) if case["bias"] else None
+        y, a = conv_transpose_ref(x, w, b, attrs, activation="relu")
+        ref = torch.relu(torch.from_numpy(_torch_special_case(x, w, b, attrs))).numpy()
+        np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12, err_msg=str(case))
+        _, a_id = conv_transpose_ref(x, w, b, attrs)
+        np.testing.assert_array_equal(a, a_id)     # the accumulator is the identity's
+    x = rng.standard_normal([1, 2, 5, 5])
+    w = rng.standard_normal([2, 3, 3, 3])
+    b = np.array([-0.5, 0.0, 0.75])
+    attrs = Attrs(strides=[2, 2], dilations=[2, 2], auto_pad="SAME_UPPER")
+    y, _ = conv_transpose_ref(x, w, b, attrs, activation="relu")
+    assert np.all(y[:, :, 0::2, :] == np.maximum(b, 0).reshape(1, 3, 1, 1))
+    with pytest.raises(ValueError):
+        conv_transpose_ref(x, w, b, attrs, activation="gelu")
+
+
 def test_against_torch_library_workload_1():
     from transposed_convolution_02_b200.workloads import make_inputs
     wl = WORKLOADS[1]

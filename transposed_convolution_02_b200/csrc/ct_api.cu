@@ -39,6 +39,7 @@ ct_status resolve(const ct_desc *d, Plan *p) {
     if (d->layout != CT_NCHW && d->layout != CT_NHWC) return CT_ERR_DTYPE;
     if (d->auto_pad < CT_AUTOPAD_NOTSET || d->auto_pad > CT_AUTOPAD_VALID) return CT_ERR_ATTR;
     if (d->algo < CT_ALGO_AUTO || d->algo > CT_ALGO_DENSE_TC_PERTAP) return CT_ERR_ATTR;
+    if (d->activation != CT_ACT_IDENTITY && d->activation != CT_ACT_RELU) return CT_ERR_ATTR;
     const int r = d->rank;
     if (d->N < 0 || d->C < 0) return CT_ERR_ATTR;
     if (d->group <= 0 || d->C % d->group != 0) return CT_ERR_CHANNELS;
@@ -59,6 +60,7 @@ ct_status resolve(const ct_desc *d, Plan *p) {
     p->Cg = d->C / d->group;
     p->Mg = mg;
     p->has_bias = d->bias_len != 0;
+    p->act = d->activation;
 
     int64_t in[3], k[3], s[3], dl[3], op[3], natural[3];
     for (int a = 0; a < r; ++a) {
@@ -342,7 +344,7 @@ const char *ct_status_string(ct_status status) {
         case CT_ERR_CHANNELS: return "channel/group arithmetic inconsistent (C, group, W dims or bias length)";
         case CT_ERR_SPAN: return "span length inconsistent (rank or attribute length)";
         case CT_ERR_DTYPE: return "dtype or layout not served";
-        case CT_ERR_ATTR: return "attribute invalid (stride, dilation, kernel, pads, output_padding, output_shape)";
+        case CT_ERR_ATTR: return "attribute invalid (stride, dilation, kernel, pads, output_padding, output_shape, activation)";
         case CT_ERR_ALIGN: return "device pointer misaligned for the chosen kernel";
         case CT_ERR_NULL: return "required pointer is NULL";
         case CT_ERR_DEVICE: return "CUDA device error (not sm_100, or launch failure)";

@@ -31,6 +31,7 @@ struct Plan {
     int64_t N, C, M, G, Cg, Mg;
     int64_t in[3], k[3], s[3], d[3], pb[3], pe[3], op[3], out[3];
     bool has_bias;
+    int act;                  // ct_activation applied after the bias
     int algo;                 // chosen ct_algo
     size_t packed_bytes;
     size_t ws_bytes;
@@ -99,5 +100,10 @@ inline ct_status launch_status() {
 }
 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// The output activation (ct_activation), applied in fp32 after the bias.
+#ifdef __CUDACC__
+__device__ __forceinline__ float apply_act(float v, int act) { return act == CT_ACT_RELU ? fmaxf(v, 0.f) : v; }
+#endif
 
 }  // namespace ct

@@ -62,7 +62,7 @@ struct HaloTables {
     int32_t TX, PU, n_units, n_groups;  // x tiles, units per (n, z, x-tile) plane
     int32_t nbuf, bufcols, SA, SB, a_bytes, a_stride, b_slot_bytes, BR;
     int32_t resident, res_rows;
-    int32_t nhwc, has_bias, dead, pair_x;
+    int32_t nhwc, has_bias, dead, pair_x, act;
     int32_t n_phases, n_items, total_rows;
     int16_t phase_r[kMaxPhases][3];
     int16_t g_phase0[kMaxGroups], g_nphase[kMaxGroups], g_item0[kMaxGroups], g_nitem[kMaxGroups];
@@ -170,13 +170,17 @@ __device__ __forceinline__ void issue4(uint32_t d, uint64_t ad, uint64_t bd, uin
     sm100::mma_f16(d, ad + 6, bd + 6, idesc, 1u);
 }
 
+template <int ACT>
 __device__ __forceinline__ void store_chunk16(__half *dst, long long stride, const uint32_t (&v)[16],
                                               const float *b, int mcount) {
 #pragma unroll
     for (int j = 0; j < 16; ++j)
-        if (j < mcount) dst[j * stride] = __float2half_rn(__uint_as_float(v[j]) + b[j]);
+        if (j < mcount) dst[j * stride] = __float2half_rn(apply_act(__uint_as_float(v[j]) + b[j], ACT));
 }
 
+// ACT: the output activation (ct_activation), fixed at compile time so that
+// the identity epilogue carries no per-element test.
+template <int ACT>
 __global__ void __launch_bounds__(kThreads, 1)
     dense_halo_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                       const __grid_constant__ HaloTables T, const __half *__restrict__ bias,
@@ -458,24 +462,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                             for (int j = 0; j < 16; ++j)
                                 if (j < mc0)
                                     *reinterpret_cast<__half2 *>(dst + j * plane) =
-                                        __floats2half2_rn(__uint_as_float(v0[j]) + bb[j],
-                                                          __uint_as_float(w0[j]) + bb[j]);
+                                        __floats2half2_rn(apply_act(__uint_as_float(v0[j]) + bb[j], ACT),
+                                                          apply_act(__uint_as_float(w0[j]) + bb[j], ACT));
                             if (two) {
                                 __half *d1 = dst + 16 * plane;
 #pragma unroll
                                 for (int j = 0; j < 16; ++j)
                                     if (j < mc1)
                                         *reinterpret_cast<__half2 *>(d1 + j * plane) =
-                                            __floats2half2_rn(__uint_as_float(v1[j]) + bb[16 + j],
-                                                              __uint_as_float(w1[j]) + bb[16 + j]);
+                                            __floats2half2_rn(apply_act(__uint_as_float(v1[j]) + bb[16 + j], ACT),
+                                                              apply_act(__uint_as_float(w1[j]) + bb[16 + j], ACT));
                             }
                         } else {
-                            store_chunk16(dst, cstride, v0, bias_s + m0, mc0);
-                            if (two) store_chunk16(dst + 16 * cstride, cstride, v1, bias_s + m0 + 16, mc1);
+                            store_chunk16<ACT>(dst, cstride, v0, bias_s + m0, mc0);
+                            if (two) store_chunk16<ACT>(dst + 16 * cstride, cstride, v1, bias_s + m0 + 16, mc1);
                             if (pair) {
                                 __half *dx = dst + xstep;   // x + 1
-                                store_chunk16(dx, cstride, w0, bias_s + m0, mc0);
-                                if (two) store_chunk16(dx + 16 * cstride, cstride, w1, bias_s + m0 + 16, mc1);
+                                store_chunk16<ACT>(dx, cstride, w0, bias_s + m0, mc0);
+                                if (two) store_chunk16<ACT>(dx + 16 * cstride, cstride, w1, bias_s + m0 + 16, mc1);
                             }
                         }
                     }
@@ -512,6 +516,7 @@ bool build_tables(const Plan &p, HaloTables &T, int Mt, int gmax_cols) {
     T.KB = (int32_t)ceil_div(p.C, 64);
     T.nhwc = p.layout == CT_NHWC;
     T.has_bias = p.has_bias;
+    T.act = p.act;
     T.Mt = Mt;
     if (T.Np > gmax_cols) return false;
     for (int a = 0; a < 3; ++a) {
@@ -792,11 +797,19 @@ ct_status dense_tc_run(const Plan &p, const void *x, const void *wp, const void 
         ct_status s2 = launch_dead_fill(p, bias, y, st);
         if (s2 != CT_OK) return s2;
     }
-    static std::atomic<int> attr_set[64];
-    if (!allow_smem(dense_halo_kernel, attr_set, kSmemBudget)) return CT_ERR_DEVICE;
     int grid = sm_count();
     if (grid > T.n_units) grid = T.n_units;
-    dense_halo_kernel<<<grid, kThreads, smem_bytes(T), st>>>(tmA, tmB, T, (const __half *)bias, (__half *)y);
+    if (T.act == CT_ACT_RELU) {
+        static std::atomic<int> attr_set[64];
+        if (!allow_smem(dense_halo_kernel<CT_ACT_RELU>, attr_set, kSmemBudget)) return CT_ERR_DEVICE;
+        dense_halo_kernel<CT_ACT_RELU><<<grid, kThreads, smem_bytes(T), st>>>(tmA, tmB, T, (const __half *)bias,
+                                                                             (__half *)y);
+    } else {
+        static std::atomic<int> attr_set[64];
+        if (!allow_smem(dense_halo_kernel<CT_ACT_IDENTITY>, attr_set, kSmemBudget)) return CT_ERR_DEVICE;
+        dense_halo_kernel<CT_ACT_IDENTITY><<<grid, kThreads, smem_bytes(T), st>>>(tmA, tmB, T,
+                                                                                 (const __half *)bias, (__half *)y);
+    }
     return launch_status();
 }
 

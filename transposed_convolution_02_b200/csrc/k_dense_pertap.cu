@@ -50,7 +50,7 @@ struct DenseTables {
     int32_t BX, BY, BZ, lbx, lby;   // tile extents in J (powers of 2), product 128
     int32_t TX, TY, TZ;             // tiles per axis
     int32_t KB, Np, stages;
-    int32_t nhwc, has_bias, dead;
+    int32_t nhwc, has_bias, dead, act;
     int32_t N, C, M;
     int32_t out[3], s[3], nJ[3];
     int16_t pair_e[kMaxPairs][3];
@@ -262,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             if (m < T.M) {
                                 float a = __uint_as_float(v[j]);
                                 if (T.has_bias) a += __half2float(bias[m]);
-                                dst[m] = __float2half_rn(a);
+                                dst[m] = __float2half_rn(apply_act(a, T.act));
                             }
                         }
                     } else {
@@ -272,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             if (m < T.M) {
                                 float a = __uint_as_float(v[j]);
                                 if (T.has_bias) a += __half2float(bias[m]);
-                                y[((long long)n * T.M + m) * plane + opos] = __float2half_rn(a);
+                                y[((long long)n * T.M + m) * plane + opos] = __float2half_rn(apply_act(a, T.act));
                             }
                         }
                     }
@@ -340,6 +340,7 @@ void dense_pertap_setup(Plan &p) {
     T.KB = (int32_t)ceil_div(p.C, 64);
     T.nhwc = p.layout == CT_NHWC;
     T.has_bias = p.has_bias;
+    T.act = p.act;
     for (int a = 0; a < 3; ++a) {
         T.out[a] = (int32_t)p.out[a];
         T.s[a] = (int32_t)p.s[a];

@@ -30,7 +30,7 @@ constexpr int kFMaxPairs = 256;
 struct F32Args {
     int32_t N, C, M, Cp, Mp;                 // Cp = C rounded to 8, Mp = M rounded to 128
     int32_t in[3], out[3], s[3], nJ[3];
-    int32_t P, tiles_p, tiles_m, n_phases, nhwc, has_bias;
+    int32_t P, tiles_p, tiles_m, n_phases, nhwc, has_bias, act;
     int32_t ph_r[kFMaxPhases][3];
     int32_t ph_q0[kFMaxPhases], ph_nq[kFMaxPhases], ph_krow[kFMaxPhases];   // first pair, pairs, packed row
     int16_t q_e[kFMaxPairs][3], q_k[kFMaxPairs][3];
@@ -155,7 +155,7 @@ __global__ void __launch_bounds__(256, 2) fp32_gemm_kernel(const __grid_constant
         for (int i = 0; i < 8; ++i) {
             const int m = m0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + i - 4);
             if (m >= A.M) continue;
-            const float v = acc[i][j] + (A.has_bias ? bias[m] : 0.f);
+            const float v = apply_act(acc[i][j] + (A.has_bias ? bias[m] : 0.f), A.act);
             if (A.nhwc)
                 y[((long long)n * plane + opos) * A.M + m] = v;
             else
@@ -211,7 +211,7 @@ __global__ void __launch_bounds__(256) fp32_dead_fill_kernel(const __grid_consta
             m = (int)(rem % A.M);
         }
         const bool live = ((m0 >> (o0 % A.s[0])) & 1) && ((m1 >> (o1 % A.s[1])) & 1) && ((m2 >> (o2 % A.s[2])) & 1);
-        if (!live) y[i] = A.has_bias ? bias[m] : 0.f;
+        if (!live) y[i] = apply_act(A.has_bias ? bias[m] : 0.f, A.act);
     }
 }
 
@@ -258,6 +258,7 @@ void fp32_setup(const Plan &p, F32Args &A) {
     }
     A.nhwc = p.layout == CT_NHWC;
     A.has_bias = p.has_bias;
+    A.act = p.act;
     int np = 0, nq = 0, krow = 0;
     for (int r0 = 0; r0 < p.s[0]; ++r0)
         for (int r1 = 0; r1 < p.s[1]; ++r1)

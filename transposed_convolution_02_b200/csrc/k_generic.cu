@@ -27,6 +27,7 @@ struct GenericArgs {
     int64_t total;
     int nhwc;
     int has_bias;
+    int act;
 };
 
 template <typename T>
@@ -101,7 +102,7 @@ __global__ void __launch_bounds__(256) generic_kernel(GenericArgs a, const T *__
             }
         }
         if (a.has_bias) acc += to_f(bias[m]);
-        y[idx] = from_f<T>(acc);
+        y[idx] = from_f<T>(apply_act(acc, a.act));
     }
 }
 
@@ -109,7 +110,7 @@ constexpr int kG32MaxS = 64;      // phases per axis
 constexpr int kG32MaxTaps = 64;   // taps per axis
 
 struct Generic32Args {
-    int32_t C, M, Cg, Mg, in_sz, k_sz, total, nhwc, has_bias;
+    int32_t C, M, Cg, Mg, in_sz, k_sz, total, nhwc, has_bias, act;
     int32_t in[3], out[3], s[3], kst[3];     // kpos = k0*kst[0] + k1*kst[1] + k2*kst[2]
     DivMagic d_out[3], d_M, d_Mg, d_s[3];
     uint8_t ph_off[3][kG32MaxS], ph_cnt[3][kG32MaxS];   // taps of phase r of axis a
@@ -179,7 +180,7 @@ __global__ void __launch_bounds__(256, 4) generic32_kernel(const __grid_constant
             }
         }
         if (a.has_bias) acc += to_f(bias[m]);
-        y[idx] = from_f<T>(acc);
+        y[idx] = from_f<T>(apply_act(acc, a.act));
     }
 }
 
@@ -198,6 +199,7 @@ bool generic32_setup(const Plan &p, Generic32Args &a) {
     a.total = (int32_t)total;
     a.nhwc = p.layout == CT_NHWC;
     a.has_bias = p.has_bias;
+    a.act = p.act;
     a.kst[2] = 1;
     a.kst[1] = (int32_t)p.k[2];
     a.kst[0] = (int32_t)(p.k[1] * p.k[2]);
@@ -256,6 +258,7 @@ ct_status generic_run(const Plan &p, const void *x, const void *wp, const void *
     a.total = p.N * p.M * numel_out(p);
     a.nhwc = p.layout == CT_NHWC;
     a.has_bias = p.has_bias;
+    a.act = p.act;
     if (a.total == 0) return CT_OK;
     const int threads = 256;
     {

@@ -61,7 +61,7 @@ struct GroupedArgs {
     int32_t N, C, M, G, Cg, Mg, KS, MT;     // KS = Cg/16 k-steps, MT = ceil(Mg/16) m-tiles
     int32_t in_y, in_x, out_y, out_x, s_y, s_x, k_y, k_x;
     int32_t nJy, nJx, JB, SR, SW, npix, emin_y, emin_x;
-    int32_t n_rb, n_seg, n_pairs, has_bias, vec8;
+    int32_t n_rb, n_seg, n_pairs, has_bias, vec8, act;
     int32_t n_live_ry, n_dead_ry, n_live_rx;
     int32_t pst;                              // bytes per re-laid pixel (2*Cg + 16)
     int32_t segp;                             // staging row pitch (halves)
@@ -115,7 +115,7 @@ __device__ __forceinline__ uint32_t bias_word(__half b) {
 // fragments are loaded two steps ahead of the MMAs that use them.  Lane pairs
 // swap half their words so that each lane stores 4 consecutive J of one
 // channel as one 16-byte piece (8-byte pieces when out_x % 8 != 0).
-template <int NSTEP>
+template <int NSTEP, int ACT>
 __device__ __forceinline__ void one_phase_rows(const GroupedArgs &A, const uint4 *__restrict__ wp,
                                                const __half *sb, uint32_t s_slab, __half *yg,
                                                long long plane, int g, int jy0, int jbv, int warp,
@@ -131,7 +131,9 @@ __device__ __forceinline__ void one_phase_rows(const GroupedArgs &A, const uint4
     const int ry = A.live_ry[0], rx = A.live_rx[0];
     const __half b0h = sb[gid], b1h = sb[gid + 8];
     const float bf0 = __half2float(b0h), bf1 = __half2float(b1h);
-    const uint32_t bw0 = __half_as_ushort(b0h), bw1 = __half_as_ushort(b1h);
+    // the other column phase's outputs: activated bias
+    const uint32_t bw0 = __half_as_ushort(__float2half_rn(apply_act(bf0, ACT)));
+    const uint32_t bw1 = __half_as_ushort(__float2half_rn(apply_act(bf1, ACT)));
     // (bias, value) order inside a 32-bit word: value high when rx == 1
     const int vsh = rx ? 16 : 0, bsh = rx ? 0 : 16;
     const bool odd = tig & 1;
@@ -191,7 +193,8 @@ __device__ __forceinline__ void one_phase_rows(const GroupedArgs &A, const uint4
             uint32_t w[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-                w[i] = ((uint32_t)__half_as_ushort(__float2half_rn(acc[nt][i])) << vsh) | ((i < 2 ? bw0 : bw1) << bsh);
+                w[i] = ((uint32_t)__half_as_ushort(__float2half_rn(apply_act(acc[nt][i], ACT))) << vsh) |
+                       ((i < 2 ? bw0 : bw1) << bsh);
             const int jx = jx0 + 8 * nt + 2 * tig;
             if (A.vec8) {
                 // even lane keeps channel gid and takes the partner's channel-gid
@@ -215,7 +218,8 @@ __device__ __forceinline__ void one_phase_rows(const GroupedArgs &A, const uint4
 // single stride phase with taps, s_x == 2, NSTEP (tap pair, k-step) steps
 // whose weight fragments and slab offsets stay in registers, and outputs
 // stored straight from the accumulators as (bias, value) pairs.
-template <int MT, int NSTEP>
+// ACT: the output activation (ct_activation), fixed at compile time.
+template <int MT, int NSTEP, int ACT>
 __global__ void __launch_bounds__(kGThreads, NSTEP > 0 ? V_OPMINB : (MT <= 2 ? 4 : 2))
     grouped_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ GroupedArgs A,
                    const __half *__restrict__ x, const uint4 *__restrict__ wp,
@@ -273,7 +277,7 @@ __global__ void __launch_bounds__(kGThreads, NSTEP > 0 ? V_OPMINB : (MT <= 2 ? 4
             if (lm >= mstep) continue;
             __half *p = yr + (long long)lm * plane;
             for (int m = lm; m < A.Mg; m += mstep, p += mstep * plane) {
-                const __half b = A.has_bias ? __ldg(bias + g * A.Mg + m) : __float2half(0.f);
+                const __half b = __float2half_rn(apply_act(A.has_bias ? __half2float(__ldg(bias + g * A.Mg + m)) : 0.f, ACT));
                 for (int c = lc; c < cols; c += 32) {
                     if (A.vec8) {
                         const uint32_t w = bias_word(b);
@@ -333,7 +337,7 @@ __global__ void __launch_bounds__(kGThreads, NSTEP > 0 ? V_OPMINB : (MT <= 2 ? 4
     __syncthreads();
 
     if constexpr (NSTEP > 0) {
-        one_phase_rows<NSTEP>(A, wp, sb, s_slab, yg, plane, g, jy0, jbv, warp, lane);
+        one_phase_rows<NSTEP, ACT>(A, wp, sb, s_slab, yg, plane, g, jy0, jbv, warp, lane);
         return;
     }
     // staging tile (over the consumed input tile): every column starts as the
@@ -344,7 +348,7 @@ __global__ void __launch_bounds__(kGThreads, NSTEP > 0 ? V_OPMINB : (MT <= 2 ? 4
         const int cpr = A.segp >> 3;
         for (int e = lane; e < MT * 16 * cpr; e += 32) {
             const int m = divq(e, A.d_cprs);
-            const uint32_t w = bias_word(sb[m]);
+            const uint32_t w = bias_word(__float2half_rn(apply_act(__half2float(sb[m]), ACT)));
             sts_v4(stg_base + (uint32_t)(m * A.segp + 8 * (e - m * cpr)) * 2, make_uint4(w, w, w, w));
         }
     }
@@ -442,8 +446,8 @@ __global__ void __launch_bounds__(kGThreads, NSTEP > 0 ? V_OPMINB : (MT <= 2 ? 4
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {
                         const uint32_t o = sl + (2 * mt + hh) * row8 + 8 * nt * colJ;
-                        sts_b16(o, __float2half_rn(acc[mt][nt][2 * hh]));
-                        sts_b16(o + colJ, __float2half_rn(acc[mt][nt][2 * hh + 1]));
+                        sts_b16(o, __float2half_rn(apply_act(acc[mt][nt][2 * hh], ACT)));
+                        sts_b16(o + colJ, __float2half_rn(apply_act(acc[mt][nt][2 * hh + 1], ACT)));
                     }
         }
         __syncwarp();
@@ -564,6 +568,7 @@ bool grouped_setup(const Plan &p, GroupedArgs &A, int jb) {
     A.k_y = (int32_t)p.k[1];
     A.k_x = (int32_t)p.k[2];
     A.has_bias = p.has_bias;
+    A.act = p.act;
     if ((long long)A.out_y * A.out_x >= (1LL << 30) || (long long)A.in_y * A.in_x >= (1LL << 30)) return false;
     int nq = 0;
     int emin_y = 1 << 20, emax_y = -(1 << 20), emin_x = 1 << 20, emax_x = -(1 << 20);
@@ -705,14 +710,21 @@ ct_status grouped_prepack(const Plan &p, const void *w, void *wp, cudaStream_t s
     return launch_status();
 }
 
+template <int MT, int NSTEP, int ACT>
+ct_status launch_grouped_act(const CUtensorMap &tm, const GroupedArgs &A, const void *x, const void *wp,
+                             const void *bias, void *y, unsigned grid, cudaStream_t st) {
+    static std::atomic<int> attr_set[64];
+    if (!allow_smem(grouped_kernel<MT, NSTEP, ACT>, attr_set, kGSmem)) return CT_ERR_DEVICE;
+    grouped_kernel<MT, NSTEP, ACT><<<grid, kGThreads, (size_t)A.smem_total, st>>>(
+        tm, A, (const __half *)x, (const uint4 *)wp, (const __half *)bias, (__half *)y);
+    return launch_status();
+}
+
 template <int MT, int NSTEP>
 ct_status launch_grouped(const CUtensorMap &tm, const GroupedArgs &A, const void *x, const void *wp,
                          const void *bias, void *y, unsigned grid, cudaStream_t st) {
-    static std::atomic<int> attr_set[64];
-    if (!allow_smem(grouped_kernel<MT, NSTEP>, attr_set, kGSmem)) return CT_ERR_DEVICE;
-    grouped_kernel<MT, NSTEP><<<grid, kGThreads, (size_t)A.smem_total, st>>>(
-        tm, A, (const __half *)x, (const uint4 *)wp, (const __half *)bias, (__half *)y);
-    return launch_status();
+    if (A.act == CT_ACT_RELU) return launch_grouped_act<MT, NSTEP, CT_ACT_RELU>(tm, A, x, wp, bias, y, grid, st);
+    return launch_grouped_act<MT, NSTEP, CT_ACT_IDENTITY>(tm, A, x, wp, bias, y, grid, st);
 }
 
 ct_status grouped_run(const Plan &p, const void *x, const void *wp, const void *bias, void *y,

@@ -53,7 +53,7 @@ struct FillArgs {
     int64_t N, M;
     int32_t out[3], s[3];
     uint64_t live[3];
-    int32_t nhwc, has_bias;
+    int32_t nhwc, has_bias, act;
 };
 
 __global__ void __launch_bounds__(256) dead_fill_kernel(const FillArgs a,
@@ -78,7 +78,7 @@ __global__ void __launch_bounds__(256) dead_fill_kernel(const FillArgs a,
         }
         const bool live = ((a.live[0] >> (o0 % a.s[0])) & 1) && ((a.live[1] >> (o1 % a.s[1])) & 1) &&
                           ((a.live[2] >> (o2 % a.s[2])) & 1);
-        if (!live) y[i] = a.has_bias ? bias[m] : __float2half(0.f);
+        if (!live) y[i] = __float2half_rn(apply_act(a.has_bias ? __half2float(bias[m]) : 0.f, a.act));
     }
 }
 
@@ -111,6 +111,7 @@ ct_status launch_dead_fill(const Plan &p, const void *bias, void *y, cudaStream_
     }
     a.nhwc = p.layout == CT_NHWC;
     a.has_bias = p.has_bias;
+    a.act = p.act;
     const long long total = p.N * p.M * numel_out(p);
     if (total == 0) return CT_OK;
     long long blocks = ceil_div(total, 256);

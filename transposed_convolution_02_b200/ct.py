@@ -53,7 +53,7 @@ class ct_desc(ctypes.Structure):
                 ("pads", ctypes.c_int64 * 6), ("output_padding", ctypes.c_int64 * 3),
                 ("has_kernel_shape", ctypes.c_int32), ("has_output_shape", ctypes.c_int32),
                 ("kernel_shape", ctypes.c_int64 * 3), ("output_shape", ctypes.c_int64 * 3),
-                ("algo", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+                ("algo", ctypes.c_int32), ("activation", ctypes.c_int32)]
 
 
 _lib = None
@@ -172,9 +172,12 @@ def ct_plan_destroy(plan):
 
 # ---- descriptor construction ----------------------------------------------
 
+ACTIVATION = {"identity": 0, "relu": 1}
+
+
 def make_desc(x_shape, w_shape, *, dtype, layout="nchw", strides=None, dilations=None,
               pads=None, output_padding=None, auto_pad="NOTSET", group=1, bias_len=0,
-              kernel_shape=None, output_shape=None, algo="auto"):
+              kernel_shape=None, output_shape=None, algo="auto", activation="identity"):
     """Fill a ct_desc from tensor shapes and README-named attributes."""
     d = ct_desc()
     r = len(x_shape) - 2
@@ -211,6 +214,7 @@ def make_desc(x_shape, w_shape, *, dtype, layout="nchw", strides=None, dilations
         for a, v in enumerate(list(output_shape)[:3]):
             d.output_shape[a] = int(v)
     d.algo = ALGO[algo]
+    d.activation = ACTIVATION.get(activation, 99)
     return d
 
 
@@ -234,7 +238,8 @@ class ConvTranspose:
 
     def __init__(self, w, x_shape, bias=None, *, layout="nchw", strides=None, dilations=None,
                  pads=None, output_padding=None, auto_pad="NOTSET", group=1,
-                 kernel_shape=None, output_shape=None, algo="auto", stream=None):
+                 kernel_shape=None, output_shape=None, algo="auto", activation="identity",
+                 stream=None):
         if not w.is_cuda:
             raise ValueError("W must be a CUDA tensor")
         self.layout = layout
@@ -243,7 +248,8 @@ class ConvTranspose:
                               strides=strides, dilations=dilations, pads=pads,
                               output_padding=output_padding, auto_pad=auto_pad, group=group,
                               bias_len=0 if bias is None else bias.numel(),
-                              kernel_shape=kernel_shape, output_shape=output_shape, algo=algo)
+                              kernel_shape=kernel_shape, output_shape=output_shape, algo=algo,
+                              activation=activation)
         self.y_shape, self.pad_begin, self.pad_end = ct_output_shape(self.desc)
         self.plan = ct_plan(self.desc)
         self.kernel = ct_plan_kernel(self.plan)
@@ -281,25 +287,26 @@ class ConvTranspose:
 
 def conv_transpose(x, w, bias=None, *, strides=None, dilations=None, pads=None,
                    output_padding=None, auto_pad="NOTSET", group=1, kernel_shape=None,
-                   output_shape=None, algo="auto"):
-    """ONNX ConvTranspose, channels-first: X[N,C,D..], W[C,M/group,k..] -> Y."""
+                   output_shape=None, algo="auto", activation="identity"):
+    """ONNX ConvTranspose, channels-first: X[N,C,D..], W[C,M/group,k..] -> Y
+    (optionally followed by the activation, identity by default)."""
     op = ConvTranspose(w, list(x.shape), bias, layout="nchw", strides=strides,
                        dilations=dilations, pads=pads, output_padding=output_padding,
                        auto_pad=auto_pad, group=group, kernel_shape=kernel_shape,
-                       output_shape=output_shape, algo=algo)
+                       output_shape=output_shape, algo=algo, activation=activation)
     return op(x)
 
 
 def conv_transpose_nhwc(x, w, bias=None, *, stride, padding, output_padding, groups,
-                        dilation, algo="auto"):
+                        dilation, activation="identity", algo="auto"):
     """Channels-last call in the form of ClikaRT::ops::conv_transpose: input
     [N, D.., C_in], weight [C_in, K.., O/groups], padding (lo, hi) per spatial
-    dim, output [N, out.., C_out]."""
+    dim, activation (identity or relu), output [N, out.., C_out]."""
     r = x.dim() - 2
     if len(padding) != 2 * r:
         raise ValueError("padding needs two entries (lo, hi) per spatial dim")
     pads = [padding[2 * a] for a in range(r)] + [padding[2 * a + 1] for a in range(r)]
     op = ConvTranspose(w, list(x.shape), bias, layout="nhwc", strides=stride,
                        dilations=dilation, pads=pads, output_padding=output_padding,
-                       group=groups, algo=algo)
+                       group=groups, algo=algo, activation=activation)
     return op(x)
