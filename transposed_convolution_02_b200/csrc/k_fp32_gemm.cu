@@ -77,24 +77,38 @@ __global__ void __launch_bounds__(256, 2) fp32_gemm_kernel(const __grid_constant
         pj[i][0] = p / A.nJ[1];
     }
     const long long in_sz = (long long)A.in[0] * A.in[1] * A.in[2];
-
-    auto load_tile = [&](int ks, float4 &ra, float (&rb)[4]) {
-        const int krow = ks * 8 + lr;             // row inside the phase's K
-        const int ql = krow / A.Cp, c = krow - ql * A.Cp;
-        ra = *reinterpret_cast<const float4 *>(wph + (size_t)krow * A.Mp + m0 + lc);
-        const int q = q0 + ql;
+    // Cp is a multiple of 8, so the 8 rows of one K stage share a tap: the
+    // tap changes every Cp/8 stages, and only then are the 4 positions' input
+    // offsets and bounds recomputed; in between the channel advances by adds.
+    const long long cstep = A.nhwc ? 1 : in_sz;          // between channels
+    long long xo[4];                                     // element offset of channel 0 at this tap
+    bool xok[4];
+    int ql = -1, c = 0;                                  // current tap of the phase, channel of row lr
+    auto set_tap = [&](int q) {
         const int e0 = A.q_e[q][0], e1 = A.q_e[q][1], e2 = A.q_e[q][2];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int iz = pj[i][0] + e0, iy = pj[i][1] + e1, ix = pj[i][2] + e2;
-            float v = 0.f;
-            if (pv[i] && c < A.C && iz >= 0 && iz < A.in[0] && iy >= 0 && iy < A.in[1] && ix >= 0 &&
-                ix < A.in[2]) {
-                const long long pos = ((long long)iz * A.in[1] + iy) * A.in[2] + ix;
-                v = A.nhwc ? x[((long long)n * in_sz + pos) * A.C + c] : x[((long long)n * A.C + c) * in_sz + pos];
-            }
-            rb[i] = v;
+            xok[i] = pv[i] && iz >= 0 && iz < A.in[0] && iy >= 0 && iy < A.in[1] && ix >= 0 && ix < A.in[2];
+            const long long pos = xok[i] ? ((long long)iz * A.in[1] + iy) * A.in[2] + ix : 0;
+            xo[i] = A.nhwc ? ((long long)n * in_sz + pos) * A.C : (long long)n * A.C * in_sz + pos;
         }
+    };
+    const float *wrow = wph + (size_t)lr * A.Mp + m0 + lc;   // this thread's W row of stage 0
+    // the next stage's operands into registers; stages are visited in order
+    auto load_tile = [&](float4 &ra, float (&rb)[4]) {
+        if (c == 0 || ql < 0) {   // stage 0 of a tap
+            ++ql;
+            set_tap(q0 + ql);
+            c = lr;
+        }
+        ra = *reinterpret_cast<const float4 *>(wrow);
+        wrow += (size_t)8 * A.Mp;
+        const bool cok = c < A.C;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) rb[i] = (cok && xok[i]) ? x[xo[i] + (long long)c * cstep] : 0.f;
+        c += 8;
+        if (c >= A.Cp) c = 0;   // the next stage starts the next tap
     };
 
     float acc[8][8];
@@ -106,7 +120,7 @@ __global__ void __launch_bounds__(256, 2) fp32_gemm_kernel(const __grid_constant
     float4 ra;
     float rb[4];
     if (ksteps > 0) {
-        load_tile(0, ra, rb);
+        load_tile(ra, rb);
         *reinterpret_cast<float4 *>(&As[0][lr][lc]) = ra;
 #pragma unroll
         for (int i = 0; i < 4; ++i) Bs[0][lr][lc + i] = rb[i];
@@ -115,7 +129,7 @@ __global__ void __launch_bounds__(256, 2) fp32_gemm_kernel(const __grid_constant
     const int ty = tid >> 4, tx = tid & 15;
     for (int ks = 0; ks < ksteps; ++ks) {
         const int cur = ks & 1;
-        if (ks + 1 < ksteps) load_tile(ks + 1, ra, rb);
+        if (ks + 1 < ksteps) load_tile(ra, rb);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
             const float4 a0 = *reinterpret_cast<const float4 *>(&As[cur][kk][ty * 4]);
