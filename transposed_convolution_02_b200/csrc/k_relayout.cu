@@ -6,44 +6,66 @@
 namespace ct {
 namespace {
 
-// channels-first -> channels-last re-layout of X (fp16), X[n][c][sp] -> Xt[n][sp][c]
+// channels-first -> channels-last re-layout of X (fp16), X[n][c][sp] -> Xt[n][sp][c].
+// A CTA moves a tile of 64 channels x 128 positions: every thread first
+// issues four 16-byte loads (four channel rows), then, after the exchange
+// through shared memory, four 16-byte stores (8 channels of one position
+// each), so each SM keeps many loads in flight and each position's 64
+// channels leave as one 128-byte run.  The 16-byte chunks of tile row r sit
+// at chunk index (chunk ^ (r >> 3) & 7), so the column reads of the eight
+// channel groups fall in distinct banks.
+
+constexpr int kRlC = 64, kRlS = 128;
 
 __global__ void __launch_bounds__(256) nchw_to_nhwc_kernel(const __half *__restrict__ x,
                                                            __half *__restrict__ xt, int C,
                                                            long long S) {
-    __shared__ __half tile[32][66];
+    __shared__ __align__(16) __half tile[kRlC][kRlS];
     const int n = blockIdx.z;
-    const int c0 = blockIdx.y * 32;
-    const long long s0 = (long long)blockIdx.x * 64;
+    const int c0 = blockIdx.y * kRlC;
+    const long long s0 = (long long)blockIdx.x * kRlS;
     const int t = threadIdx.x;
+    const bool vec = (S & 7) == 0;
     {
-        const int cl = t >> 3, sv = t & 7;
-        const int c = c0 + cl;
+        // 16 threads per channel row (16 x 8 positions), 16 rows per pass
+        const int cl = t >> 4, sv = t & 15;
         const long long s = s0 + sv * 8;
-        const __half *src = x + ((long long)n * C + c) * S + s;
-        if (c < C && (S & 7) == 0 && s + 8 <= S) {
-            uint4 v = *reinterpret_cast<const uint4 *>(src);
-            const __half2 *h = reinterpret_cast<const __half2 *>(&v);
+        uint4 v[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-                *reinterpret_cast<__half2 *>(&tile[cl][sv * 8 + 2 * j]) = h[j];
-        } else {
+        for (int r = 0; r < 4; ++r) {
+            const int c = c0 + cl + 16 * r;
+            const __half *src = x + ((long long)n * C + c) * S + s;
+            if (vec && c < C && s + 8 <= S) {
+                v[r] = __ldg(reinterpret_cast<const uint4 *>(src));
+            } else {
+                __align__(16) __half h[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-                tile[cl][sv * 8 + j] = (c < C && s + j < S) ? src[j] : __float2half(0.f);
+                for (int j = 0; j < 8; ++j) h[j] = (c < C && s + j < S) ? src[j] : __float2half(0.f);
+                v[r] = *reinterpret_cast<const uint4 *>(h);
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const int row = cl + 16 * r;
+            *reinterpret_cast<uint4 *>(&tile[row][(sv ^ ((row >> 3) & 7)) * 8]) = v[r];
         }
     }
     __syncthreads();
     {
-        const int sl = t >> 2, cv = t & 3;
-        const long long s = s0 + sl;
+        // 8 threads per position (8 x 8 channels), 32 positions per pass
+        const int sl = t >> 3, cv = t & 7;
         const int c = c0 + cv * 8;
-        if (s < S && c < C) {
-            __align__(16) __half v[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) v[j] = tile[cv * 8 + j][sl];
-            *reinterpret_cast<uint4 *>(xt + ((long long)n * S + s) * C + c) =
-                *reinterpret_cast<const uint4 *>(v);
+        for (int r = 0; r < 4; ++r) {
+            const int sp = sl + 32 * r;
+            const long long s = s0 + sp;
+            if (s < S && c < C) {
+                __align__(16) __half v[8];
+                const int col = (((sp >> 3) ^ cv) << 3) | (sp & 7);   // rows cv*8 + j: (row >> 3) & 7 == cv
+#pragma unroll
+                for (int j = 0; j < 8; ++j) v[j] = tile[cv * 8 + j][col];
+                *reinterpret_cast<uint4 *>(xt + ((long long)n * S + s) * C + c) = *reinterpret_cast<const uint4 *>(v);
+            }
         }
     }
 }
@@ -86,7 +108,8 @@ __global__ void __launch_bounds__(256) dead_fill_kernel(const FillArgs a,
 
 ct_status launch_nchw_to_nhwc_f16(const Plan &p, const void *x, void *xt, cudaStream_t st) {
     const long long S = numel_in(p);
-    dim3 grid((unsigned)ceil_div(S, 64), (unsigned)ceil_div(p.C, 32), (unsigned)p.N);
+    if (ceil_div(p.C, kRlC) > 65535 || p.N > 65535 || ceil_div(S, kRlS) > 0x7fffffffLL) return CT_ERR_UNSUPPORTED;
+    dim3 grid((unsigned)ceil_div(S, kRlS), (unsigned)ceil_div(p.C, kRlC), (unsigned)p.N);
     nchw_to_nhwc_kernel<<<grid, 256, 0, st>>>((const __half *)x, (__half *)xt, (int)p.C, S);
     return launch_status();
 }
