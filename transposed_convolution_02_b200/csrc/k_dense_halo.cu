@@ -623,6 +623,15 @@ bool build_tables(const Plan &p, HaloTables &T, int Mt, int gmax_cols) {
         for (auto &q : pairs) offs.push_back({q.e0, q.e1, q.e2});
         std::sort(offs.begin(), offs.end());
         offs.erase(std::unique(offs.begin(), offs.end()), offs.end());
+        // offsets shared by more phases first: their phases are then all
+        // untouched and merge into one wide item instead of several narrow ones
+        auto nph = [&](const std::array<int, 3> &e) {
+            int c = 0;
+            for (auto &q : pairs) c += (q.e0 == e[0] && q.e1 == e[1] && q.e2 == e[2]);
+            return c;
+        };
+        std::stable_sort(offs.begin(), offs.end(),
+                         [&](const std::array<int, 3> &a, const std::array<int, 3> &b) { return nph(a) > nph(b); });
         std::vector<char> touched(np, 0);
         T.g_item0[g] = (int16_t)ni;
         int brow = 0;
