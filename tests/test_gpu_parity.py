@@ -14,6 +14,7 @@ from cases import random_case
 from parity import (check_close, draw_case, full_parity, gpu_run, sampled_parity, to_oracle,
                     attrs_from)
 from oracle import conv_transpose_ref
+from transposed_convolution_02_b200 import ct
 from transposed_convolution_02_b200.workloads import WORKLOADS, make_inputs
 
 pytestmark = pytest.mark.gpu
@@ -272,3 +273,40 @@ def test_fp32_gemm_random_sweep(layout):
         case["w_shape"][1] = m
         full_parity(case, torch.float32, 11000 + i, layout, algo="fp32_gemm",
                     expect_kernel="fp32_gemm")
+
+
+@pytest.mark.parametrize("algo,dtype,layout,case", [
+    ("dense_tc", torch.float16, "nchw", dict(x_shape=[2, 64, 9, 20], w_shape=[64, 72, 4, 4], strides=[2, 2],
+                                             pads=[1, 1, 1, 1], bias=True)),
+    ("dense_tc", torch.float16, "nhwc", dict(x_shape=[2, 64, 9, 20], w_shape=[64, 72, 4, 4], strides=[2, 2],
+                                             pads=[1, 1, 1, 1], bias=True)),
+    ("dense_tc_pertap", torch.float16, "nchw", dict(x_shape=[2, 32, 6, 5], w_shape=[32, 40, 3, 3],
+                                                    strides=[2, 2], pads=[1, 1, 1, 1], bias=True)),
+    ("grouped", torch.float16, "nchw", dict(x_shape=[2, 64, 7, 9], w_shape=[64, 24, 2, 2], strides=[2, 2],
+                                            group=2, bias=True)),
+    ("fp32_gemm", torch.float32, "nchw", dict(x_shape=[2, 24, 40], w_shape=[24, 40, 4], strides=[4],
+                                              pads=[1, 2], bias=True)),
+    ("generic", torch.float16, "nchw", dict(x_shape=[2, 6, 7], w_shape=[6, 4, 3], strides=[2], bias=True)),
+])
+def test_bias_off_16_byte_boundary(algo, dtype, layout, case):
+    """A bias that starts one element past a 16-byte boundary (a view into a
+    larger tensor): the kernels that read the bias in 16-byte pieces take
+    their element-wise path instead."""
+    x, w, b = draw_case(case, dtype, 95, layout)
+    store = torch.zeros(b.numel() + 1, dtype=dtype, device="cuda")
+    store[1:] = b.cuda()
+    bview = store[1:]
+    assert bview.data_ptr() % 16 != 0
+    op = ct.ConvTranspose(w.cuda(), list(x.shape), bview, layout=layout, strides=case["strides"],
+                          dilations=case.get("dilations"), pads=case.get("pads"),
+                          group=case.get("group", 1), algo=algo)
+    assert op.kernel == algo, op.kernel
+    y = torch.full(op.y_shape, float("nan"), dtype=dtype, device="cuda")
+    op(x.cuda(), out=y)
+    torch.cuda.synchronize()
+    xa, wa, ba = to_oracle(x, w, b, layout)
+    ref, absacc = conv_transpose_ref(xa, wa, ba, attrs_from(case))
+    if layout == "nhwc":
+        ref = np.moveaxis(ref, 1, -1)
+        absacc = np.moveaxis(absacc, 1, -1)
+    check_close(y, ref, absacc, dtype, "unaligned bias %s %s" % (algo, layout))

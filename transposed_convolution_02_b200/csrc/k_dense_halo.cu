@@ -407,6 +407,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int out0 = T.out[0], out1 = T.out[1], out2 = T.out[2];
         const int s0 = T.s[0], s1 = T.s[1], s2 = T.s[2];
         const int nJ1 = T.nJ[1], nJ2 = T.nJ[2];
+        const bool has_bias = T.has_bias;
+        const bool bias_vec = has_bias && (reinterpret_cast<uintptr_t>(bias) & 15) == 0;
         const long long plane = (long long)out0 * out1 * out2;
         const long long cstride = nhwc ? 1 : plane;        // between channels
         const long long xstep = nhwc ? (long long)M : 1;   // between x positions
@@ -453,11 +455,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                         __half *dst = base + (long long)m0 * cstride;
                         if (!nhwc && pair) {
                             // both x phases of a channel are adjacent: one half2 per channel
+                            // bias through the read-only global path: shared-memory
+                            // reads here wait behind the next unit's tile loads
                             float bb[32];
+                            if (bias_vec && m0 + 32 <= M) {
 #pragma unroll
-                            for (int j = 0; j < 8; ++j)
-                                *reinterpret_cast<float4 *>(&bb[4 * j]) =
-                                    *reinterpret_cast<const float4 *>(&bias_s[m0 + 4 * j]);
+                                for (int j = 0; j < 4; ++j) {
+                                    const uint4 h = __ldg(reinterpret_cast<const uint4 *>(bias + m0) + j);
+                                    const __half2 *h2 = reinterpret_cast<const __half2 *>(&h);
+#pragma unroll
+                                    for (int q = 0; q < 4; ++q) {
+                                        const float2 f = __half22float2(h2[q]);
+                                        bb[8 * j + 2 * q] = f.x;
+                                        bb[8 * j + 2 * q + 1] = f.y;
+                                    }
+                                }
+                            } else if (!has_bias) {
+#pragma unroll
+                                for (int j = 0; j < 32; ++j) bb[j] = 0.f;
+                            } else {   // the last, partial chunk of channels, or an unaligned bias
+#pragma unroll
+                                for (int j = 0; j < 32; ++j) bb[j] = bias_s[m0 + j];
+                            }
 #pragma unroll
                             for (int j = 0; j < 16; ++j)
                                 if (j < mc0)
