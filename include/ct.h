@@ -85,8 +85,12 @@ typedef enum ct_algo {
     CT_ALGO_DENSE_TC = 2,  /* fp16 group-1 phase GEMM on tcgen05 tensor cores */
     CT_ALGO_FP32_GEMM = 3, /* fp32 group-1 register-tiled FFMA phase GEMM */
     CT_ALGO_GROUPED = 4,   /* fp16 grouped phase kernel (mma.sync), small per-group slabs */
-    CT_ALGO_DENSE_TC_PERTAP = 5 /* fp16 group-1 tcgen05 phase GEMM, one input load per tap
-                                   (the general fallback of CT_ALGO_DENSE_TC) */
+    CT_ALGO_DENSE_TC_PERTAP = 5, /* fp16 group-1 tcgen05 phase GEMM, one input load per tap
+                                    (the general fallback of CT_ALGO_DENSE_TC) */
+    CT_ALGO_DENSE_TC_PAIR = 6    /* fp16 group-1 phase GEMM with one or two spatial axes and
+                                    channels-first layout, each MMA spanning the two SMs of a
+                                    CTA pair (tcgen05 cta_group::2); the workspace holds a
+                                    zero-padded channels-last copy of X */
 } ct_algo;
 
 /* Activation applied to every output after the bias (ClikaRT::ops::

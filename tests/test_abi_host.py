@@ -151,7 +151,7 @@ def test_workload_shapes_and_plan(wid):
     assert ys == list(wl.y_shape)
     plan = ct.ct_plan(d)
     try:
-        assert ct.ct_plan_kernel(plan) in ("generic", "dense_tc", "fp32_gemm", "grouped")
+        assert ct.ct_plan_kernel(plan) in ("generic", "dense_tc", "dense_tc_pair", "fp32_gemm", "grouped")
         assert ct.ct_prepacked_weight_bytes(plan) > 0
         assert ct.ct_workspace_bytes(plan) >= 0
     finally:

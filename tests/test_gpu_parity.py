@@ -287,6 +287,8 @@ def test_fp32_gemm_random_sweep(layout):
     ("fp32_gemm", torch.float32, "nchw", dict(x_shape=[2, 24, 40], w_shape=[24, 40, 4], strides=[4],
                                               pads=[1, 2], bias=True)),
     ("generic", torch.float16, "nchw", dict(x_shape=[2, 6, 7], w_shape=[6, 4, 3], strides=[2], bias=True)),
+    ("dense_tc_pair", torch.float16, "nchw", dict(x_shape=[2, 64, 9, 20], w_shape=[64, 72, 4, 4],
+                                                  strides=[2, 2], pads=[1, 1, 1, 1], bias=True)),
 ])
 def test_bias_off_16_byte_boundary(algo, dtype, layout, case):
     """A bias that starts one element past a 16-byte boundary (a view into a
@@ -310,3 +312,57 @@ def test_bias_off_16_byte_boundary(algo, dtype, layout, case):
         ref = np.moveaxis(ref, 1, -1)
         absacc = np.moveaxis(absacc, 1, -1)
     check_close(y, ref, absacc, dtype, "unaligned bias %s %s" % (algo, layout))
+
+
+def _pair_case(rng):
+    case = random_case(rng, max_rank=2, groups=(1,), max_cg=1, max_mg=1,
+                       lim_in={1: 700, 2: 40}, lim_k={1: 9, 2: 5})
+    c = int(rng.choice([8, 16, 24, 64, 72, 136, 256]))
+    m = int(rng.choice([1, 7, 16, 33, 64, 100, 128, 200, 256]))
+    case["x_shape"][1] = c
+    case["w_shape"][0] = c
+    case["w_shape"][1] = m
+    return case
+
+
+def test_dense_tc_pair_random_sweep():
+    """fp16 group-1 channels-first shapes with one or two spatial axes on the
+    CTA-pair tcgen05 kernel: strides/dilations up to 4, negative and
+    asymmetric pads, output_padding, M not a multiple of 16 (up to 256), C
+    spanning partial 64-channel blocks, phases without taps.  Shapes whose
+    padded input run exceeds the kernel's tile are refused at plan time."""
+    rng = np.random.default_rng(600)
+    ran = 0
+    for i in range(70):
+        case = _pair_case(rng)
+        try:
+            full_parity(case, torch.float16, 9000 + i, "nchw", algo="dense_tc_pair",
+                        expect_kernel="dense_tc_pair")
+        except ct.CtError as e:
+            assert e.status == 9, e   # CT_ERR_UNSUPPORTED from ct_plan
+            continue
+        ran += 1
+    assert ran >= 30, ran
+
+
+@pytest.mark.parametrize("case", [
+    # the 2-D decoder's attributes on a smaller image: several units per image, ragged tail
+    dict(x_shape=[3, 256, 21, 23], w_shape=[256, 128, 4, 4], strides=[2, 2], pads=[1, 1, 1, 1], bias=True),
+    # M = 256 (one phase per accumulator buffer) and M = 200 (Np 208)
+    dict(x_shape=[2, 64, 11, 13], w_shape=[64, 256, 4, 4], strides=[2, 2], pads=[1, 1, 1, 1], bias=True),
+    dict(x_shape=[2, 72, 9, 17], w_shape=[72, 200, 3, 3], strides=[2, 2], pads=[1, 1, 1, 1],
+         output_padding=[1, 1], bias=True),
+    # stride 1 (a plain 3x3 convolution with tap-reversed weights), no bias
+    dict(x_shape=[2, 64, 30, 30], w_shape=[64, 64, 3, 3], strides=[1, 1], pads=[1, 1, 1, 1]),
+    # taps only on odd outputs: the rest is the bias
+    dict(x_shape=[2, 32, 9, 10], w_shape=[32, 48, 3, 3], strides=[2, 2], dilations=[2, 2],
+         auto_pad="SAME_UPPER", bias=True),
+    # one spatial axis: a long fp16 vocoder-style upsample
+    dict(x_shape=[2, 64, 3000], w_shape=[64, 32, 16], strides=[8], pads=[4, 4], bias=True),
+    # stride 3, odd output width (no paired x phases), C = 8
+    dict(x_shape=[1, 8, 15, 19], w_shape=[8, 24, 5, 5], strides=[3, 3], pads=[2, 1, 0, 2], bias=True),
+])
+def test_dense_tc_pair_cases(case):
+    full_parity(case, torch.float16, 77, "nchw", algo="dense_tc_pair", expect_kernel="dense_tc_pair")
+    full_parity(dict(case, activation="relu"), torch.float16, 78, "nchw", algo="dense_tc_pair",
+                expect_kernel="dense_tc_pair")

@@ -38,7 +38,7 @@ ct_status resolve(const ct_desc *d, Plan *p) {
     if (d->dtype != CT_F32 && d->dtype != CT_F16) return CT_ERR_DTYPE;
     if (d->layout != CT_NCHW && d->layout != CT_NHWC) return CT_ERR_DTYPE;
     if (d->auto_pad < CT_AUTOPAD_NOTSET || d->auto_pad > CT_AUTOPAD_VALID) return CT_ERR_ATTR;
-    if (d->algo < CT_ALGO_AUTO || d->algo > CT_ALGO_DENSE_TC_PERTAP) return CT_ERR_ATTR;
+    if (d->algo < CT_ALGO_AUTO || d->algo > CT_ALGO_DENSE_TC_PAIR) return CT_ERR_ATTR;
     if (d->activation != CT_ACT_IDENTITY && d->activation != CT_ACT_RELU) return CT_ERR_ATTR;
     const int r = d->rank;
     if (d->N < 0 || d->C < 0) return CT_ERR_ATTR;
@@ -146,7 +146,11 @@ void choose(Plan *p) {
     // tiny problems: one gather launch beats any tiled kernel's set-up
     const double flop = 2.0 * p->N * p->C * p->Mg * numel_in(*p) * numel_k(*p);
     if (want == CT_ALGO_AUTO && flop < 1e7) return;
-    if ((want == CT_ALGO_AUTO || want == CT_ALGO_DENSE_TC) && dense_tc_supports(*p)) {
+    if ((want == CT_ALGO_AUTO || want == CT_ALGO_DENSE_TC_PAIR) && dense_pair_supports(*p)) {
+        p->algo = CT_ALGO_DENSE_TC_PAIR;
+    } else if (want == CT_ALGO_DENSE_TC_PAIR) {
+        p->algo = -1;
+    } else if ((want == CT_ALGO_AUTO || want == CT_ALGO_DENSE_TC) && dense_tc_supports(*p)) {
         p->algo = CT_ALGO_DENSE_TC;
     } else if ((want == CT_ALGO_AUTO || want == CT_ALGO_DENSE_TC || want == CT_ALGO_DENSE_TC_PERTAP) &&
                dense_pertap_supports(*p)) {
@@ -239,6 +243,11 @@ ct_status ct_plan(const ct_desc *desc, ct_plan_t **out) {
             p->packed_bytes = dense_tc_packed_bytes(*p);
             p->ws_bytes = dense_tc_ws_bytes(*p);
             break;
+        case CT_ALGO_DENSE_TC_PAIR:
+            dense_pair_setup(*p);
+            p->packed_bytes = dense_pair_packed_bytes(*p);
+            p->ws_bytes = dense_pair_ws_bytes(*p);
+            break;
         case CT_ALGO_DENSE_TC_PERTAP:
             dense_pertap_setup(*p);
             p->packed_bytes = dense_pertap_packed_bytes(*p);
@@ -263,6 +272,7 @@ const char *ct_plan_kernel(const ct_plan_t *plan) {
     switch (reinterpret_cast<const Plan *>(plan)->algo) {
         case CT_ALGO_DENSE_TC: return "dense_tc";
         case CT_ALGO_DENSE_TC_PERTAP: return "dense_tc_pertap";
+        case CT_ALGO_DENSE_TC_PAIR: return "dense_tc_pair";
         case CT_ALGO_FP32_GEMM: return "fp32_gemm";
         case CT_ALGO_GROUPED: return "grouped";
         default: return "generic";
@@ -299,6 +309,7 @@ ct_status ct_prepack_weights(const ct_plan_t *plan, const void *w, void *w_packe
     switch (p.algo) {
         case CT_ALGO_DENSE_TC: return dense_tc_prepack(p, w, w_packed, s);
         case CT_ALGO_DENSE_TC_PERTAP: return dense_pertap_prepack(p, w, w_packed, s);
+        case CT_ALGO_DENSE_TC_PAIR: return dense_pair_prepack(p, w, w_packed, s);
         case CT_ALGO_GROUPED: return grouped_prepack(p, w, w_packed, s);
         case CT_ALGO_FP32_GEMM: return fp32_gemm_prepack(p, w, w_packed, s);
         default: return generic_prepack(p, w, w_packed, s);
@@ -330,6 +341,7 @@ ct_status ct_run(const ct_plan_t *plan, const void *x, const void *w_packed, con
     switch (p.algo) {
         case CT_ALGO_DENSE_TC: return dense_tc_run(p, x, w_packed, bias, y, workspace, s);
         case CT_ALGO_DENSE_TC_PERTAP: return dense_pertap_run(p, x, w_packed, bias, y, workspace, s);
+        case CT_ALGO_DENSE_TC_PAIR: return dense_pair_run(p, x, w_packed, bias, y, workspace, s);
         case CT_ALGO_GROUPED: return grouped_run(p, x, w_packed, bias, y, s);
         case CT_ALGO_FP32_GEMM: return fp32_gemm_run(p, x, w_packed, bias, y, s);
         default: return generic_run(p, x, w_packed, bias, y, s);

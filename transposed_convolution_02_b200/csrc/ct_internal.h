@@ -79,6 +79,14 @@ ct_status dense_tc_prepack(const Plan &p, const void *w, void *wp, cudaStream_t 
 ct_status dense_tc_run(const Plan &p, const void *x, const void *wp, const void *bias, void *y,
                        void *ws, cudaStream_t st);
 
+bool dense_pair_supports(const Plan &p);
+size_t dense_pair_packed_bytes(const Plan &p);
+size_t dense_pair_ws_bytes(const Plan &p);
+void dense_pair_setup(Plan &p);
+ct_status dense_pair_prepack(const Plan &p, const void *w, void *wp, cudaStream_t st);
+ct_status dense_pair_run(const Plan &p, const void *x, const void *wp, const void *bias, void *y,
+                         void *ws, cudaStream_t st);
+
 bool fp32_gemm_supports(const Plan &p);
 void fp32_gemm_plan(Plan &p);
 size_t fp32_gemm_packed_bytes(const Plan &p);

@@ -28,7 +28,7 @@ CT_F32, CT_F16 = 0, 1
 CT_NCHW, CT_NHWC = 0, 1
 AUTOPAD = {"NOTSET": 0, "SAME_UPPER": 1, "SAME_LOWER": 2, "VALID": 3}
 ALGO = {"auto": 0, "generic": 1, "dense_tc": 2, "fp32_gemm": 3, "grouped": 4,
-        "dense_tc_pertap": 5}
+        "dense_tc_pertap": 5, "dense_tc_pair": 6}
 
 EXPORTED = ["ct_output_shape", "ct_plan", "ct_plan_kernel", "ct_plan_launches",
             "ct_prepacked_weight_bytes",
