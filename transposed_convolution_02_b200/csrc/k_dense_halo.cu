@@ -22,7 +22,10 @@
 //  * A unit covers Mt tiles of 128 positions, so each weight tile feeds Mt
 //    MMAs; weights stay resident in shared memory when they all fit.
 // Warps: 0 loads input tiles, 1 issues MMAs, 2-3 load weights, 4-7 drain TMEM
-// (bias from shared memory, fp16 rounding, paired x phases stored as half2).
+// (bias, fp16 rounding; paired x phases stored as half2 channels-first, 16
+// channels as two 16-byte vectors channels-last).  More epilogue warps were
+// measured slower here: the register cap of a larger block costs the 3-D
+// upsample more than the extra store parallelism gains.
 #include <cuda.h>
 
 #include <algorithm>
@@ -41,6 +44,7 @@ constexpr int kMaxPhases = 64;
 constexpr int kMaxGroups = 64;
 constexpr int kMaxItems = 512;
 constexpr int kThreads = 256;
+constexpr int kEpiSets = (kThreads / 32 - 4) / 4;   // epilogue warps per TMEM lane quarter
 constexpr int kSmemBudget = 227 * 1024;
 
 struct Item {
@@ -170,6 +174,26 @@ __device__ __forceinline__ void issue4(uint32_t d, uint64_t ad, uint64_t bd, uin
     sm100::mma_f16(d, ad + 6, bd + 6, idesc, 1u);
 }
 
+// 16 consecutive channels of one channels-last position: two 16-byte stores
+// when the row is whole and aligned, else element by element.
+template <int ACT>
+__device__ __forceinline__ void store_row16(__half *dst, const uint32_t (&v)[16], const float *b, int mcount) {
+    if (mcount == 16 && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+        uint4 q[2];
+        __half2 *h = reinterpret_cast<__half2 *>(q);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            h[j] = __floats2half2_rn(apply_act(__uint_as_float(v[2 * j]) + b[2 * j], ACT),
+                                     apply_act(__uint_as_float(v[2 * j + 1]) + b[2 * j + 1], ACT));
+        reinterpret_cast<uint4 *>(dst)[0] = q[0];
+        reinterpret_cast<uint4 *>(dst)[1] = q[1];
+    } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            if (j < mcount) dst[j] = __float2half_rn(apply_act(__uint_as_float(v[j]) + b[j], ACT));
+    }
+}
+
 template <int ACT>
 __device__ __forceinline__ void store_chunk16(__half *dst, long long stride, const uint32_t (&v)[16],
                                               const float *b, int mcount) {
@@ -224,7 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull + 8 * b, 1);
-            mbar_init(tempty + 8 * b, 128);
+            mbar_init(tempty + 8 * b, kThreads / 32 - 4);   // one arrival per epilogue warp
         }
         mbar_init(bres, 1);
         mbar_init(mdone, 1);
@@ -327,82 +351,81 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = first; j < ib; ++j)
                 if ((j & 1) == me) mbar_wait(fullB + 8 * (j % SB), (j / SB) & 1, err, 5);
         }
-    } else if (warp == 1 && lane == 0) {
+    } else if (warp == 1) {
         // ---------------- MMA issue ----------------
+        // The whole warp walks the loop, so every descriptor it computes is
+        // warp-uniform (items are read from the kernel parameters with uniform
+        // indices, ring positions advance by counters); one elected lane
+        // issues the MMAs and commits.  A single-lane loop cannot keep narrow
+        // MMAs back to back.
+        const bool issuer = elect_one();
         bool ok = true;
-        if (resident) ok = mbar_wait(bres, 0, err, 6);
-        int ia = 0, local = 0;
-        uint32_t sb_slot = 0, sb_phase = 0;   // weight ring position of the next item
+        if (resident) ok = __all_sync(0xffffffffu, mbar_wait(bres, 0, err, 6));
+        int local = 0;
+        uint32_t sa_slot = 0, sa_phase = 0, sb_slot = 0, sb_phase = 0;
         for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++local) {
             const Unit U = decode_unit(G, u);
-            const SGroup gr = groups_s[U.g];
+            const int i0 = T.g_item0[U.g], i1 = i0 + T.g_nitem[U.g];
+            const int gbrow = T.g_brow[U.g], grows = T.g_rows_kb[U.g];
             const int buf = nbuf == 2 ? (local & 1) : 0;
             const int use = nbuf == 2 ? (local >> 1) : local;
-            if (use > 0 && !mbar_wait(tempty + 8 * buf, (use - 1) & 1, err, 7)) break;
+            if (use > 0) ok = __all_sync(0xffffffffu, mbar_wait(tempty + 8 * buf, (use - 1) & 1, err, 7));
+            if (!ok) break;
             tc_fence_after();
             const uint32_t dbase = tmem_base + buf * bufcols;
-            const int gcols = gr.nphase * Np;
+            const uint32_t mstep = (uint32_t)(T.g_nphase[U.g] * Np);
             const int rel = U.F0 - U.y0 * HX;   // row of the unit's first position in the tile
-            for (int kb = 0; kb < KB && ok; ++kb, ++ia) {
-                const int sa = ia % SA;
-                if (!mbar_wait(fullA + 8 * sa, (ia / SA) & 1, err, 8)) {
-                    ok = false;
-                    break;
-                }
+            for (int kb = 0; kb < KB; ++kb) {
+                ok = __all_sync(0xffffffffu, mbar_wait(fullA + 8 * sa_slot, sa_phase, err, 8));
+                if (!ok) break;
                 tc_fence_after();
-                const uint32_t a_addr = smem_u32(sA + (size_t)sa * a_stride) + (uint32_t)rel * 128;
-                const uint32_t bres_base = smem_u32(sB) + (uint32_t)((gr.brow + kb * gr.rows_kb) * 128);
-                const int i0 = gr.item0, i1 = gr.item0 + gr.nitem;
-                const uint32_t mstep = (uint32_t)gcols;
-                if (resident) {
-                    // weights resident: nothing to wait for between items
-                    for (int it = i0; it < i1; ++it) {
-                        const SItem I = items_s[it];
-                        const uint64_t bd = desc_kmajor_sw128(bres_base + (uint32_t)I.brow * 128);
-                        const uint64_t ad = desc_kmajor_sw128(a_addr + (uint32_t)I.shift * 128);
-                        const uint32_t idesc = idesc_f16_f32(128, I.n);
-                        const uint32_t d = dbase + I.tcol;
-                        const uint32_t acc0 = (kb == 0 && I.first) ? 0u : 1u;
-                        issue4(d, ad, bd, idesc, acc0);
-                        if (Mt > 1) issue4(d + mstep, ad + 1024, bd, idesc, acc0);   // +128 rows
-                    }
-                } else {
-                    // Shared-memory reads of this thread wait behind the MMAs'
-                    // operand reads, so the next item's entry is fetched before
-                    // the current item's MMAs are issued, and the ring slot and
-                    // phase advance by counters instead of divisions.
-                    SItem In = items_s[i0];
-                    for (int it = i0; it < i1; ++it) {
-                        const SItem I = In;
-                        if (it + 1 < i1) In = items_s[it + 1];
-                        if (!mbar_wait(fullB + 8 * sb_slot, sb_phase, err, 9)) {
-                            ok = false;
-                            break;
-                        }
+                const uint32_t a_addr = smem_u32(sA) + sa_slot * (uint32_t)a_stride + (uint32_t)rel * 128;
+                const uint32_t bres_base = smem_u32(sB) + (uint32_t)((gbrow + kb * grows) * 128);
+                for (int it = i0; it < i1; ++it) {
+                    uint32_t b_addr;
+                    if (resident) {
+                        b_addr = bres_base + (uint32_t)T.item[it].brow * 128;
+                    } else {
+                        ok = __all_sync(0xffffffffu, mbar_wait(fullB + 8 * sb_slot, sb_phase, err, 9));
+                        if (!ok) break;
                         tc_fence_after();
-                        const uint64_t bd = desc_kmajor_sw128(smem_u32(sB) + sb_slot * (uint32_t)b_slot);
-                        const uint64_t ad = desc_kmajor_sw128(a_addr + (uint32_t)I.shift * 128);
-                        const uint32_t idesc = idesc_f16_f32(128, I.n);
-                        const uint32_t d = dbase + I.tcol;
-                        const uint32_t acc0 = (kb == 0 && I.first) ? 0u : 1u;
+                        b_addr = smem_u32(sB) + sb_slot * (uint32_t)b_slot;
+                    }
+                    const uint64_t bd = desc_kmajor_sw128(b_addr);
+                    const uint64_t ad = desc_kmajor_sw128(a_addr + (uint32_t)T.item[it].shift * 128);
+                    const uint32_t idesc = idesc_f16_f32(128, T.item[it].n);
+                    const uint32_t d = dbase + (uint32_t)T.item[it].tcol;
+                    const uint32_t acc0 = (kb == 0 && T.item[it].first) ? 0u : 1u;
+                    if (issuer) {
                         issue4(d, ad, bd, idesc, acc0);
                         if (Mt > 1) issue4(d + mstep, ad + 1024, bd, idesc, acc0);   // +128 rows
-                        mma_commit(emptyB + 8 * sb_slot);
-                        if (++sb_slot == (uint32_t)SB) {
-                            sb_slot = 0;
-                            sb_phase ^= 1u;
-                        }
+                        if (!resident) mma_commit(emptyB + 8 * sb_slot);
+                    }
+                    __syncwarp();
+                    if (!resident && ++sb_slot == (uint32_t)SB) {
+                        sb_slot = 0;
+                        sb_phase ^= 1u;
                     }
                 }
-                mma_commit(emptyA + 8 * sa);
+                if (!ok) break;
+                if (issuer) mma_commit(emptyA + 8 * sa_slot);
+                __syncwarp();
+                if (++sa_slot == (uint32_t)SA) {
+                    sa_slot = 0;
+                    sa_phase ^= 1u;
+                }
             }
-            mma_commit(tfull + 8 * buf);
+            if (!ok) break;
+            if (issuer) mma_commit(tfull + 8 * buf);
+            __syncwarp();
         }
-        mma_commit(mdone);
+        if (issuer) mma_commit(mdone);
+        __syncwarp();
         mbar_wait(mdone, 0, err, 10);
     } else if (warp >= 4) {
         // ---------------- epilogue ----------------
-        const int lane_base = 32 * (warp & 3);
+        const int lane_base = 32 * (warp & 3);   // the TMEM lane quarter this warp may read
+        const int eh = (warp - 4) >> 2;           // first 32-channel chunk of this warp's set
         const int p = lane_base + lane;
         const int out0 = T.out[0], out1 = T.out[1], out2 = T.out[2];
         const int s0 = T.s[0], s1 = T.s[1], s2 = T.s[2];
@@ -415,14 +438,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         int local = 0;
         for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++local) {
             const Unit U = decode_unit(G, u);
-            const SGroup gr = groups_s[U.g];
             const int buf = nbuf == 2 ? (local & 1) : 0;
             const int use = nbuf == 2 ? (local >> 1) : local;
             if (!mbar_wait(tfull + 8 * buf, use & 1, err, 11)) break;
             tc_fence_after();
             const uint32_t dbase = tmem_base + ((uint32_t)lane_base << 16) + buf * bufcols;
-            const int gcols = gr.nphase * Np;
-            const int ph0 = gr.phase0, ph1 = ph0 + gr.nphase;
+            const int gcols = T.g_nphase[U.g] * Np;
+            const int ph0 = T.g_phase0[U.g], ph1 = ph0 + T.g_nphase[U.g];
             for (int mt = 0; mt < Mt; ++mt) {
                 const int F = U.F0 + mt * 128 + p;
                 const int jxl = F % HX;
@@ -430,17 +452,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int Jx = U.tx * BXt + jxl;
                 const bool pos_ok = jxl < BXt && Jx < nJ2 && Jy < nJ1;
                 for (int ph = ph0; ph < ph1;) {
-                    const int r0 = phr_s[3 * ph], r1 = phr_s[3 * ph + 1], r2 = phr_s[3 * ph + 2];
+                    const int r0 = T.phase_r[ph][0], r1 = T.phase_r[ph][1], r2 = T.phase_r[ph][2];
                     const int oz = s0 * U.jz + r0;
                     const int oy = s1 * Jy + r1;
                     const int ox = s2 * Jx + r2;
                     const bool valid = pos_ok && oz < out0 && oy < out1 && ox < out2;
-                    const bool pair = pair_x && ph + 1 < ph1 && (r2 & 1) == 0 && phr_s[3 * ph + 5] == r2 + 1 &&
-                                      phr_s[3 * ph + 4] == r1 && phr_s[3 * ph + 3] == r0;
+                    const bool pair = pair_x && ph + 1 < ph1 && (r2 & 1) == 0 && T.phase_r[ph + 1][2] == r2 + 1 &&
+                                      T.phase_r[ph + 1][1] == r1 && T.phase_r[ph + 1][0] == r0;
                     const long long opos = ((long long)oz * out1 + oy) * out2 + ox;
                     const uint32_t col0 = dbase + mt * gcols + (ph - ph0) * Np;
                     __half *base = nhwc ? y + ((long long)U.n * plane + opos) * M : y + (long long)U.n * M * plane + opos;
-                    for (int m0 = 0; m0 < Np; m0 += 32) {
+                    for (int m0 = 32 * eh; m0 < Np; m0 += 32 * kEpiSets) {
                         uint32_t v0[16], v1[16], w0[16], w1[16];
                         const bool two = m0 + 16 < Np;
                         tmem_ld16(col0 + m0, v0);
@@ -492,6 +514,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                                             __floats2half2_rn(apply_act(__uint_as_float(v1[j]) + bb[16 + j], ACT),
                                                               apply_act(__uint_as_float(w1[j]) + bb[16 + j], ACT));
                             }
+                        } else if (nhwc) {
+                            float bb[32];
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) bb[j] = bias_s[m0 + j];
+                            store_row16<ACT>(dst, v0, bb, mc0);
+                            if (two) store_row16<ACT>(dst + 16, v1, bb + 16, mc1);
+                            if (pair) {
+                                __half *dx = dst + xstep;   // x + 1
+                                store_row16<ACT>(dx, w0, bb, mc0);
+                                if (two) store_row16<ACT>(dx + 16, w1, bb + 16, mc1);
+                            }
                         } else {
                             store_chunk16<ACT>(dst, cstride, v0, bias_s + m0, mc0);
                             if (two) store_chunk16<ACT>(dst + 16 * cstride, cstride, v1, bias_s + m0 + 16, mc1);
@@ -506,7 +539,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             tc_fence_before();
-            mbar_arrive(tempty + 8 * buf);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty + 8 * buf);
         }
     }
     __syncthreads();
