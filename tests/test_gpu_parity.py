@@ -315,8 +315,8 @@ def test_bias_off_16_byte_boundary(algo, dtype, layout, case):
 
 
 def _pair_case(rng):
-    case = random_case(rng, max_rank=2, groups=(1,), max_cg=1, max_mg=1,
-                       lim_in={1: 700, 2: 40}, lim_k={1: 9, 2: 5})
+    case = random_case(rng, max_rank=3, groups=(1,), max_cg=1, max_mg=1,
+                       lim_in={1: 700, 2: 40, 3: 12}, lim_k={1: 9, 2: 5, 3: 3})
     c = int(rng.choice([8, 16, 24, 64, 72, 136, 256]))
     m = int(rng.choice([1, 7, 16, 33, 64, 100, 128, 200, 256]))
     case["x_shape"][1] = c
@@ -326,11 +326,11 @@ def _pair_case(rng):
 
 
 def test_dense_tc_pair_random_sweep():
-    """fp16 group-1 channels-first shapes with one or two spatial axes on the
-    CTA-pair tcgen05 kernel: strides/dilations up to 4, negative and
+    """fp16 group-1 channels-first shapes with one to three spatial axes on
+    the CTA-pair tcgen05 kernel: strides/dilations up to 4, negative and
     asymmetric pads, output_padding, M not a multiple of 16 (up to 256), C
     spanning partial 64-channel blocks, phases without taps.  Shapes whose
-    padded input run exceeds the kernel's tile are refused at plan time."""
+    padded input runs exceed the kernel's tile are refused at plan time."""
     rng = np.random.default_rng(600)
     ran = 0
     for i in range(70):
@@ -361,6 +361,12 @@ def test_dense_tc_pair_random_sweep():
     dict(x_shape=[2, 64, 3000], w_shape=[64, 32, 16], strides=[8], pads=[4, 4], bias=True),
     # stride 3, odd output width (no paired x phases), C = 8
     dict(x_shape=[1, 8, 15, 19], w_shape=[8, 24, 5, 5], strides=[3, 3], pads=[2, 1, 0, 2], bias=True),
+    # the 3-D upsample's attributes on a smaller volume (two input slices per unit)
+    dict(x_shape=[2, 64, 6, 9, 11], w_shape=[64, 32, 3, 3, 3], strides=[2, 2, 2], pads=[1, 1, 1, 1, 1, 1],
+         output_padding=[1, 1, 1]),
+    # 3-D, stride 1 along z (three input slices), M = 40
+    dict(x_shape=[1, 16, 5, 7, 6], w_shape=[16, 40, 3, 2, 2], strides=[1, 2, 2], pads=[1, 0, 0, 1, 1, 0],
+         bias=True),
 ])
 def test_dense_tc_pair_cases(case):
     full_parity(case, torch.float16, 77, "nchw", algo="dense_tc_pair", expect_kernel="dense_tc_pair")

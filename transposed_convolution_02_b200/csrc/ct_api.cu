@@ -146,7 +146,8 @@ void choose(Plan *p) {
     // tiny problems: one gather launch beats any tiled kernel's set-up
     const double flop = 2.0 * p->N * p->C * p->Mg * numel_in(*p) * numel_k(*p);
     if (want == CT_ALGO_AUTO && flop < 1e7) return;
-    if ((want == CT_ALGO_AUTO || want == CT_ALGO_DENSE_TC_PAIR) && dense_pair_supports(*p)) {
+    if (((want == CT_ALGO_AUTO && dense_pair_preferred(*p)) || want == CT_ALGO_DENSE_TC_PAIR) &&
+        dense_pair_supports(*p)) {
         p->algo = CT_ALGO_DENSE_TC_PAIR;
     } else if (want == CT_ALGO_DENSE_TC_PAIR) {
         p->algo = -1;

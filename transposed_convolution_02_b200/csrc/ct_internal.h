@@ -80,6 +80,7 @@ ct_status dense_tc_run(const Plan &p, const void *x, const void *wp, const void 
                        void *ws, cudaStream_t st);
 
 bool dense_pair_supports(const Plan &p);
+bool dense_pair_preferred(const Plan &p);   // auto selection: where it measured fastest
 size_t dense_pair_packed_bytes(const Plan &p);
 size_t dense_pair_ws_bytes(const Plan &p);
 void dense_pair_setup(Plan &p);
