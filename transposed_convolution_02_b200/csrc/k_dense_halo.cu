@@ -294,6 +294,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == 0 && lane == 0) {
         // ---------------- input tiles ----------------
+        // X (or its channels-last copy) may be the previous grid's output
+        griddep_wait();
         int ia = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
@@ -317,6 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if ((warp == 2 || warp == 3) && lane == 0) {
         // ---------------- weight tiles: two issuing warps, alternate ring items ----------------
         const int me = warp - 2;
+        griddep_wait();   // the packed weights may be the previous grid's output
         if (resident) {
             if (me == 0) {
                 mbar_arrive_expect_tx(bres, (uint32_t)res_rows * 128);
@@ -861,16 +864,33 @@ ct_status dense_tc_run(const Plan &p, const void *x, const void *wp, const void 
     }
     int grid = sm_count();
     if (grid > T.n_units) grid = T.n_units;
+    // programmatic dependent launch: the set-up overlaps the tail of the grid
+    // before; both producers wait for it before loading
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem_bytes(T);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const __half *b = (const __half *)bias;
+    __half *yy = (__half *)y;
+    cudaError_t e;
     if (T.act == CT_ACT_RELU) {
         static std::atomic<int> attr_set[64];
         if (!allow_smem(dense_halo_kernel<CT_ACT_RELU>, attr_set, kSmemBudget)) return CT_ERR_DEVICE;
-        dense_halo_kernel<CT_ACT_RELU><<<grid, kThreads, smem_bytes(T), st>>>(tmA, tmB, T, (const __half *)bias,
-                                                                             (__half *)y);
+        e = cudaLaunchKernelEx(&cfg, dense_halo_kernel<CT_ACT_RELU>, tmA, tmB, T, b, yy);
     } else {
         static std::atomic<int> attr_set[64];
         if (!allow_smem(dense_halo_kernel<CT_ACT_IDENTITY>, attr_set, kSmemBudget)) return CT_ERR_DEVICE;
-        dense_halo_kernel<CT_ACT_IDENTITY><<<grid, kThreads, smem_bytes(T), st>>>(tmA, tmB, T,
-                                                                                 (const __half *)bias, (__half *)y);
+        e = cudaLaunchKernelEx(&cfg, dense_halo_kernel<CT_ACT_IDENTITY>, tmA, tmB, T, b, yy);
+    }
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return CT_ERR_DEVICE;
     }
     return launch_status();
 }

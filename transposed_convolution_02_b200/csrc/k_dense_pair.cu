@@ -183,6 +183,7 @@ __global__ void __launch_bounds__(256) nchw_to_padded_kernel(const __half *__res
     const long long P2 = (long long)HY * HX;
     const long long P = g.HZ * P2;
     const int t = threadIdx.x;
+    sm100::griddep_launch_dependents();   // the pair kernel may set up while this one runs
     if ((int)blockIdx.x < g.halo_blocks) {
         // zero halo of image n, channels [c0, c0 + 64), spread over the halo blocks
         const int c0 = blockIdx.y * kPadC;
@@ -347,6 +348,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
 
     if (warp == 0 && lane == 0) {
         // ---------------- input runs (both CTAs; rank 0 expects both halves) ----------------
+        // the padded copy is the previous grid's output: wait for it here
+        // only, after the set-up and while the weight loads go out
+        griddep_wait();
         int ia = 0;
         bool ok = true;
         for (int u = cid; u < n_units && ok; u += ncl) {
@@ -842,7 +846,24 @@ ct_status launch_pair(const PairTables &T, const CUtensorMap &tmA, const CUtenso
     const size_t smem = pair_launch_smem(T);
     int pairs = resident_pairs(dense_pair_kernel<ACT>, (int)smem);
     if (pairs > T.n_units) pairs = T.n_units;
-    dense_pair_kernel<ACT><<<2 * pairs, kPThreads, smem, st>>>(tmA, tmB, tmBs, T, (const __half *)bias, (__half *)y);
+    // programmatic dependent launch: the kernel's set-up overlaps the tail of
+    // the re-layout (or the bias fill) before it; the input producer waits
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * pairs, 1, 1);
+    cfg.blockDim = dim3(kPThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const __half *b = (const __half *)bias;
+    __half *yy = (__half *)y;
+    if (cudaLaunchKernelEx(&cfg, dense_pair_kernel<ACT>, tmA, tmB, tmBs, T, b, yy) != cudaSuccess) {
+        cudaGetLastError();
+        return CT_ERR_DEVICE;
+    }
     return launch_status();
 }
 

@@ -2,6 +2,7 @@
 // channels-last re-layout of fp16 X, and the bias fill of outputs that no
 // tap reaches (their stride phase has no tap on some axis).
 #include "ct_internal.h"
+#include "sm100.cuh"
 
 namespace ct {
 namespace {
@@ -21,6 +22,7 @@ __global__ void __launch_bounds__(256) nchw_to_nhwc_kernel(const __half *__restr
                                                            __half *__restrict__ xt, int C,
                                                            long long S) {
     __shared__ __align__(16) __half tile[kRlC][kRlS];
+    sm100::griddep_launch_dependents();   // the tensor-core kernel may set up while this one runs
     const int n = blockIdx.z;
     const int c0 = blockIdx.y * kRlC;
     const long long s0 = (long long)blockIdx.x * kRlS;

@@ -148,6 +148,16 @@ __device__ __forceinline__ bool elect_one() {
     return pred != 0;
 }
 
+// ---- programmatic dependent launch --------------------------------------------
+// Let the next grid in the stream start launching (its CTAs are placed as
+// resources free up; it must still wait before reading this grid's output).
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Wait until the grids this one depends on have completed and their memory
+// is visible (a no-op when the launch carried no programmatic dependency).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---- CTA pairs (clusters of two) ------------------------------------------------
 // A pair's tcgen05 MMA (cta_group::2) spans both SMs: rank 0 issues it, each
 // CTA supplies its half of A (128 rows) and of B (N/2 rows) from its own
