@@ -67,9 +67,21 @@ def load_peaks():
                 sm_max_mhz=1965.0, source="fallback")
 
 
-def roofline_for(wl, seconds_per_launch, peaks, sms):
+# Nominal dense TF32 : BF16 tensor rates of a B200 (1.1 : 2.25 PFLOP/s): the
+# TF32 peak is the measured BF16 peak times this ratio.
+TF32_PER_BF16 = 1.1 / 2.25
+
+
+def roofline_for(wl, seconds_per_launch, peaks, sms, kernel=None):
     """Bound and achieved rate of the workload's dominant kernel."""
     flop, nbytes = workload_numbers(wl)
+    if wl.dtype == torch.float32 and kernel == "dense_tc_pair":
+        # 3xTF32 on the tensor cores: three TF32 MMAs per fp32 product, so the
+        # algorithmic fp32 rate is bounded by a third of the TF32 peak
+        peak = peaks["tc_tflops"] * TF32_PER_BF16 / 3
+        a = flop / seconds_per_launch / 1e12
+        return dict(bound="tensor", achieved=a, peak=peak, unit="TFLOP/s", frac=a / peak,
+                    peak_note="3xTF32: measured bf16 peak x %.3f (nominal TF32/BF16) / 3" % TF32_PER_BF16)
     if wl.dtype == torch.float32:
         # FP32 FFMA peak: SMs x 128 lanes x 2 flop x max SM clock
         peak = sms * 128 * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12
@@ -430,7 +442,7 @@ def main():
     ms, info = time_device(wl, device, args.steps, args.warmup, l2, dist_max, sampler)
     ms, value = aggregate(flop, ms, args.steps, world, dist_max)
     sec_per_step = ms / 1e3 / args.steps
-    roof = roofline_for(wl, sec_per_step, peaks, props.multi_processor_count)
+    roof = roofline_for(wl, sec_per_step, peaks, props.multi_processor_count, info["kernel"])
     roof["peak_source"] = peaks["source"] + " (burst)"
     annotate_roofline(roof, args.workload, info["kernel"], info["launches_per_step"])
     roof["per_call_us"] = sec_per_step * 1e6
@@ -451,7 +463,7 @@ def main():
             if dist_max is not None:
                 oms = dist_max("max", oms)
             osec = oms / 1e3 / osteps
-            oroof = roofline_for(owl, osec, peaks, props.multi_processor_count)
+            oroof = roofline_for(owl, osec, peaks, props.multi_processor_count, oinfo["kernel"])
             annotate_roofline(oroof, wid, oinfo["kernel"], oinfo["launches_per_step"])
             others[str(wid)] = {"workload": owl.name, "kernel": oinfo["kernel"],
                                 "us_per_step": osec * 1e6, "tflops": ofl / osec / 1e12,

@@ -372,3 +372,41 @@ def test_dense_tc_pair_cases(case):
     full_parity(case, torch.float16, 77, "nchw", algo="dense_tc_pair", expect_kernel="dense_tc_pair")
     full_parity(dict(case, activation="relu"), torch.float16, 78, "nchw", algo="dense_tc_pair",
                 expect_kernel="dense_tc_pair")
+
+
+@pytest.mark.parametrize("case", [
+    # the 1-D vocoder's attributes on a shorter signal
+    dict(x_shape=[2, 64, 300], w_shape=[64, 48, 16], strides=[8], pads=[4, 4], bias=True),
+    # 2-D stride 2 with M = 40 and C = 36 (a partial 32-channel block)
+    dict(x_shape=[2, 36, 9, 13], w_shape=[36, 40, 4, 4], strides=[2, 2], pads=[1, 1, 1, 1], bias=True),
+    # 3-D, odd output width, no bias
+    dict(x_shape=[1, 32, 4, 5, 7], w_shape=[32, 24, 3, 3, 3], strides=[2, 2, 2], pads=[1, 1, 1, 1, 1, 1]),
+    # taps only on odd outputs
+    dict(x_shape=[2, 16, 7, 8], w_shape=[16, 32, 3, 3], strides=[2, 2], dilations=[2, 2],
+         auto_pad="SAME_UPPER", bias=True),
+])
+def test_dense_tc_pair_fp32(case):
+    """The CTA-pair kernel on fp32 operands (3xTF32: high and low TF32 parts,
+    three MMAs per step) within the fp32 tolerance."""
+    full_parity(case, torch.float32, 79, "nchw", algo="dense_tc_pair", expect_kernel="dense_tc_pair")
+    full_parity(dict(case, activation="relu"), torch.float32, 80, "nchw", algo="dense_tc_pair",
+                expect_kernel="dense_tc_pair")
+
+
+def test_dense_tc_pair_fp32_random_sweep():
+    """fp32 group-1 channels-first shapes with one to three spatial axes on the
+    3xTF32 CTA-pair kernel, compared with the fp64 oracle at the fp32
+    tolerance."""
+    rng = np.random.default_rng(610)
+    ran = 0
+    for i in range(40):
+        case = _pair_case(rng)
+        case["x_shape"][1] = case["w_shape"][0] = int(rng.choice([4, 12, 32, 36, 64, 100]))
+        try:
+            full_parity(case, torch.float32, 9500 + i, "nchw", algo="dense_tc_pair",
+                        expect_kernel="dense_tc_pair")
+        except ct.CtError as e:
+            assert e.status == 9, e
+            continue
+        ran += 1
+    assert ran >= 15, ran

@@ -59,6 +59,9 @@ struct PItem {
 
 struct PairTables {
     int32_t N, C, M, Np, KB;
+    // f32: fp32 operands as a TF32 high part and its remainder (3xTF32: three
+    // MMAs per step), 32 channels per 128-byte row; otherwise fp16, 64 channels
+    int32_t f32, cpb, parts;            // parts: 2 (high, low) for f32, else 1
     int32_t in[3], out[3], s[3], pb[3], d[3], k[3], nJ[3];   // axes z, y, x
     int32_t emin[3], HX, HY, HZ;
     int32_t n_slices, slice_rows, chunk_rows, n_chunks, a_bytes, a_stride;
@@ -70,8 +73,9 @@ struct PairTables {
     int32_t g_brow[kPMaxGroups], g_rows_kb[kPMaxGroups];
     int16_t g_chunk0[kPMaxGroups], g_nchunk[kPMaxGroups];
     // a chunk: consecutive items of a group whose weights one barrier covers;
-    // inside one channel block its rows are [row0, row0 + half) for rank 0,
-    // then [row0 + half, row0 + 2 half) for rank 1
+    // inside one channel block its rows are [row0, row0 + parts*half) for
+    // rank 0, then the same count for rank 1; with two parts a rank's block
+    // holds the high parts (half rows), then the low parts
     int16_t c_item0[kPMaxChunks], c_nitem[kPMaxChunks];
     int32_t c_row0[kPMaxChunks], c_half[kPMaxChunks];
     PItem item[kPMaxItems];
@@ -82,20 +86,25 @@ __device__ int g_dense_pair_err;
 const PairTables &ptables(const Plan &p) { return *reinterpret_cast<const PairTables *>(p.aux.data()); }
 
 // ---------------------------------------------------------------------------
-// weight pre-pack: rows of every group, channel block, chunk and rank in the
-// order the kernel loads them; a row holds 64 input channels of one output
-// channel m of one phase, W[kb*64 + cc][m][kz][ky][kx] at the phase's taps for the
-// item's offset, zero outside C and M.  Rows [0, n/2) of an item's N columns
-// feed the pair's rank 0, rows [n/2, n) rank 1.
+// weight pre-pack: rows of every group, channel block, chunk, rank (and part)
+// in the order the kernel loads them; a row holds the 64 (fp16) or 32 (fp32)
+// input channels of one output channel m of one phase at one channel block,
+// W[kb*cpb + cc][m][kz][ky][kx] at the phase's tap for the item's offset, zero
+// outside C and M.  Rows [0, n/2) of an item's N columns feed the pair's
+// rank 0, rows [n/2, n) rank 1.  For fp32 a weight w is stored as its TF32
+// high part h (low 13 mantissa bits cleared) and the remainder w - h.
 
+__device__ __forceinline__ float tf32_high(float v) { return __uint_as_float(__float_as_uint(v) & 0xffffe000u); }
+
+template <typename E>
 __global__ void __launch_bounds__(256) pair_prepack_kernel(const __grid_constant__ PairTables T,
-                                                           const __half *__restrict__ w,
-                                                           __half *__restrict__ wp) {
-    const long long total = (long long)T.total_rows * 64;
+                                                           const E *__restrict__ w, E *__restrict__ wp) {
+    const int cpb = T.cpb, parts = T.parts;
+    const long long total = (long long)T.total_rows * cpb;
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
          i += (long long)gridDim.x * blockDim.x) {
-        const int cc = (int)(i & 63);
-        const int row = (int)(i >> 6);
+        const int cc = (int)(i % cpb);
+        const int row = (int)(i / cpb);
         int g = 0;
         while (g + 1 < T.n_groups && row >= T.g_brow[g + 1]) ++g;
         const int rg = row - T.g_brow[g];
@@ -104,18 +113,21 @@ __global__ void __launch_bounds__(256) pair_prepack_kernel(const __grid_constant
         int c = T.g_chunk0[g];
         const int c1 = T.g_chunk0[g] + T.g_nchunk[g];
         while (c + 1 < c1 && rk >= T.c_row0[c + 1]) ++c;
+        const int half = T.c_half[c];
         const int r2 = rk - T.c_row0[c];
-        const int rank = r2 >= T.c_half[c] ? 1 : 0;
-        const int r3 = r2 - rank * T.c_half[c];
+        const int rank = r2 >= parts * half ? 1 : 0;
+        const int r3 = r2 - rank * parts * half;
+        const int part = r3 >= half ? 1 : 0;   // 1: the remainder (fp32 only)
+        const int r4 = r3 - part * half;
         int it = T.c_item0[c];
         const int i1 = T.c_item0[c] + T.c_nitem[c];
-        while (it + 1 < i1 && r3 >= T.item[it + 1].crow) ++it;
+        while (it + 1 < i1 && r4 >= T.item[it + 1].crow) ++it;
         const PItem &I = T.item[it];
-        const int rr = rank * (I.n / 2) + (r3 - I.crow);
+        const int rr = rank * (I.n / 2) + (r4 - I.crow);
         const int ph = I.phase0 + rr / T.Np;
         const int m = rr % T.Np;
-        const int ci = kb * 64 + cc;
-        __half v = __float2half(0.f);
+        const int ci = kb * cpb + cc;
+        float v = 0.f;
         if (ci < T.C && m < T.M) {
             long long kpos = 0;
             bool ok = true;
@@ -125,9 +137,10 @@ __global__ void __launch_bounds__(256) pair_prepack_kernel(const __grid_constant
                 ok = ok && num % T.d[a] == 0 && ka >= 0 && ka < T.k[a];
                 kpos = kpos * T.k[a] + ka;
             }
-            if (ok) v = w[((long long)ci * T.M + m) * ((long long)T.k[0] * T.k[1] * T.k[2]) + kpos];
+            if (ok) v = (float)w[((long long)ci * T.M + m) * ((long long)T.k[0] * T.k[1] * T.k[2]) + kpos];
         }
-        wp[i] = v;
+        if (parts == 2) v = part ? v - tf32_high(v) : tf32_high(v);
+        wp[i] = (E)v;
     }
 }
 
@@ -271,6 +284,110 @@ __global__ void __launch_bounds__(256) nchw_to_padded_kernel(const __half *__res
     }
 }
 
+// fp32: X -> two padded channels-last planes, the TF32 high parts and the
+// remainders (3xTF32 operands); tiles of 32 channels x 128 positions, halo
+// blocks as above.  The shared tile has a pitch of 129 words, so the column
+// reads of a warp fall in 32 different banks.
+constexpr int kPadC32 = 32;
+
+__global__ void __launch_bounds__(256) nchw_to_padded_f32_kernel(const float *__restrict__ x,
+                                                                 float *__restrict__ xh, float *__restrict__ xl,
+                                                                 const PadGeo g) {
+    const int n = blockIdx.z;
+    const int C = g.C, H = g.H, W = g.W, HY = g.HY, HX = g.HX;
+    const long long HW = (long long)H * W;
+    const long long S = g.D * HW;
+    const long long P2 = (long long)HY * HX;
+    const long long P = g.HZ * P2;
+    const int t = threadIdx.x;
+    sm100::griddep_launch_dependents();   // the pair kernel may set up while this one runs
+    if ((int)blockIdx.x < g.halo_blocks) {
+        const int c0 = blockIdx.y * kPadC32;
+        const int c4 = (min(kPadC32, C - c0)) >> 2;
+        const HaloCount h = halo_count(g);
+        const long long work = h.n_all * c4;
+        for (long long q = (long long)blockIdx.x * blockDim.x + t; q < work; q += (long long)g.halo_blocks * blockDim.x) {
+            const long long k = q / c4;
+            const int cc = (int)(q - k * c4);
+            long long pos;
+            if (k < h.n_zt || k >= h.n_zt + h.n_zm) {
+                pos = k < h.n_zt ? k : (long long)h.zmid_end * P2 + (k - h.n_zt - h.n_zm);
+            } else {
+                const int kk = (int)(k - h.n_zt);
+                const int zq = kk / h.h2;
+                const int k2 = kk - zq * h.h2;
+                int yp, xq;
+                if (k2 < h.n_top) {
+                    yp = k2 / HX;
+                    xq = k2 - yp * HX;
+                } else if (k2 < h.n_top + h.n_mid) {
+                    const int r = (k2 - h.n_top) / h.lr, j = (k2 - h.n_top) - r * h.lr;
+                    yp = h.top + r;
+                    xq = j < h.left ? j : h.right0 + (j - h.left);
+                } else {
+                    const int k3 = k2 - h.n_top - h.n_mid;
+                    yp = h.mid_end + k3 / HX;
+                    xq = k3 - (k3 / HX) * HX;
+                }
+                pos = (long long)(h.ztop + zq) * P2 + (long long)yp * HX + xq;
+            }
+            const long long off = ((long long)n * P + pos) * C + c0 + cc * 4;
+            *reinterpret_cast<float4 *>(xh + off) = make_float4(0.f, 0.f, 0.f, 0.f);
+            *reinterpret_cast<float4 *>(xl + off) = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        return;
+    }
+    __shared__ float tile[kPadC32][kPadS + 1];
+    const int c0 = blockIdx.y * kPadC32;
+    const long long s0 = (long long)(blockIdx.x - g.halo_blocks) * kPadS;
+    const bool vec = (S & 3) == 0;
+    {
+        // 8 threads per channel row, 16 positions each
+        const int cl = t >> 3, sv = t & 7;
+        const int c = c0 + cl;
+        const long long s = s0 + sv * 16;
+        const float *src = x + ((long long)n * C + c) * S + s;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            float4 v;
+            if (vec && c < C && s + 4 * j + 4 <= S) {
+                v = __ldg(reinterpret_cast<const float4 *>(src) + j);
+            } else {
+                const long long b = s + 4 * j;
+                v.x = (c < C && b < S) ? src[4 * j] : 0.f;
+                v.y = (c < C && b + 1 < S) ? src[4 * j + 1] : 0.f;
+                v.z = (c < C && b + 2 < S) ? src[4 * j + 2] : 0.f;
+                v.w = (c < C && b + 3 < S) ? src[4 * j + 3] : 0.f;
+            }
+            float *d = &tile[cl][sv * 16 + 4 * j];
+            d[0] = v.x;
+            d[1] = v.y;
+            d[2] = v.z;
+            d[3] = v.w;
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        // a task: one position and 4 channels
+        const int task = t + 256 * r;
+        const int q = task & 7, sp = task >> 3;
+        const long long s = s0 + sp;
+        const int c = c0 + 4 * q;
+        if (s >= S || c >= C) continue;
+        const int iz = (int)s / (int)HW;   // S < 2^31
+        const int rem = (int)s - iz * (int)HW;
+        const int iy = rem / W, ix = rem - iy * W;
+        const int zp = iz + g.oz, yp = iy + g.oy, xq = ix + g.ox;
+        if (zp < 0 || zp >= g.HZ || yp < 0 || yp >= HY || xq < 0 || xq >= HX) continue;
+        const float4 v = make_float4(tile[4 * q][sp], tile[4 * q + 1][sp], tile[4 * q + 2][sp], tile[4 * q + 3][sp]);
+        const float4 hi = make_float4(tf32_high(v.x), tf32_high(v.y), tf32_high(v.z), tf32_high(v.w));
+        const long long off = ((long long)n * P + zp * P2 + (long long)yp * HX + xq) * C + c;
+        *reinterpret_cast<float4 *>(xh + off) = hi;
+        *reinterpret_cast<float4 *>(xl + off) = make_float4(v.x - hi.x, v.y - hi.y, v.z - hi.z, v.w - hi.w);
+    }
+}
+
 // ---------------------------------------------------------------------------
 // A unit: image n, output slice jz, group g, pair positions [pu*256, +256) of
 // the slice; rank r of the pair owns [pu*256 + 128*r, +128).  Units are
@@ -283,12 +400,49 @@ __device__ __forceinline__ float act_f(float v) {
     return apply_act(v, ACT);
 }
 
-template <int ACT>
+// Output stores of the epilogue for fp16 and fp32 elements.
+__device__ __forceinline__ void st_pair(__half *p, float a, float b) {
+    *reinterpret_cast<__half2 *>(p) = __floats2half2_rn(a, b);
+}
+__device__ __forceinline__ void st_pair(float *p, float a, float b) { *reinterpret_cast<float2 *>(p) = make_float2(a, b); }
+__device__ __forceinline__ void st_one(__half *p, float a) { *p = __float2half_rn(a); }
+__device__ __forceinline__ void st_one(float *p, float a) { *p = a; }
+// 32 bias values from global memory (16-byte aligned source)
+__device__ __forceinline__ void ld_bias32(const __half *b, float (&bb)[32]) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint4 h = __ldg(reinterpret_cast<const uint4 *>(b) + j);
+        const __half2 *h2 = reinterpret_cast<const __half2 *>(&h);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float2 f = __half22float2(h2[q]);
+            bb[8 * j + 2 * q] = f.x;
+            bb[8 * j + 2 * q + 1] = f.y;
+        }
+    }
+}
+__device__ __forceinline__ void ld_bias32(const float *b, float (&bb)[32]) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const float4 f = __ldg(reinterpret_cast<const float4 *>(b) + j);
+        bb[4 * j] = f.x;
+        bb[4 * j + 1] = f.y;
+        bb[4 * j + 2] = f.z;
+        bb[4 * j + 3] = f.w;
+    }
+}
+
+// E: the element type, __half (fp16 MMAs) or float (3xTF32: a TF32 high part
+// and its remainder for both operands, hi*hi + hi*lo + lo*hi per step).
+template <int ACT, typename E>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
     dense_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                       const __grid_constant__ CUtensorMap tmBs, const __grid_constant__ PairTables T,
-                      const __half *__restrict__ bias, __half *__restrict__ y) {
+                      const E *__restrict__ bias, E *__restrict__ y) {
     using namespace sm100;
+    constexpr bool kF32 = sizeof(E) == 4;
+    constexpr int kParts = kF32 ? 2 : 1;
+    constexpr int kCpb = kF32 ? 32 : 64;   // channels per 128-byte row
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -332,7 +486,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
         prefetch_tmap(&tmBs);
     }
     for (int m = threadIdx.x; m < ((Np + 31) & ~31); m += kPThreads)
-        bias_s[m] = (T.has_bias && m < M) ? __half2float(bias[m]) : 0.f;
+        bias_s[m] = (T.has_bias && m < M) ? (float)bias[m] : 0.f;
     if (warp == 1) {
         tmem_alloc_pair(smem_u32(tmem_slot), 512);
         tmem_relinquish_pair();
@@ -365,12 +519,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
                     ok = false;
                     break;
                 }
-                if (rank == 0) mbar_arrive_expect_tx(fullA + 8 * s, 2u * (uint32_t)a_bytes);
+                if (rank == 0) mbar_arrive_expect_tx(fullA + 8 * s, 2u * kParts * (uint32_t)a_bytes);
                 const uint32_t dst = smem_u32(sA + (size_t)s * a_stride);
-                for (int dz = 0; dz < n_slices; ++dz)
-                    for (int ch = 0; ch < n_chunks; ++ch)
-                        tma_load_2d_pair(dst + (uint32_t)((dz * slice_rows + ch * chunk_rows) * 128), &tmA,
-                                         fullA0 + 8 * s, kb * 64, (int)(row0 + dz * slice_pos + ch * chunk_rows));
+                for (int part = 0; part < kParts; ++part)
+                    for (int dz = 0; dz < n_slices; ++dz)
+                        for (int ch = 0; ch < n_chunks; ++ch)
+                            tma_load_3d_pair(dst + (uint32_t)(part * a_bytes + (dz * slice_rows + ch * chunk_rows) * 128),
+                                             &tmA, fullA0 + 8 * s, kb * kCpb,
+                                             (int)(row0 + dz * slice_pos + ch * chunk_rows), part);
             }
         }
         // rank 0's last barrier phases cover both CTAs' copies in flight
@@ -395,13 +551,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
                         ok = false;
                         break;
                     }
-                    const int half = T.c_half[c];
-                    if (rank == 0) mbar_arrive_expect_tx(fullB + 8 * s, 2u * (uint32_t)half * 128);
+                    const int rows = kParts * T.c_half[c];   // this rank's rows of the chunk
+                    if (rank == 0) mbar_arrive_expect_tx(fullB + 8 * s, 2u * (uint32_t)rows * 128);
                     const uint32_t dst = smem_u32(sB + (size_t)s * b_slot);
-                    const int row = rowbase + T.c_row0[c] + (int)rank * half;
+                    const int row = rowbase + T.c_row0[c] + (int)rank * rows;
                     int r = 0;
-                    for (; r + BR <= half; r += BR) tma_load_2d_pair(dst + (uint32_t)r * 128, &tmB, fullB0 + 8 * s, 0, row + r);
-                    for (; r < half; r += BRs) tma_load_2d_pair(dst + (uint32_t)r * 128, &tmBs, fullB0 + 8 * s, 0, row + r);
+                    for (; r + BR <= rows; r += BR) tma_load_2d_pair(dst + (uint32_t)r * 128, &tmB, fullB0 + 8 * s, 0, row + r);
+                    for (; r < rows; r += BRs) tma_load_2d_pair(dst + (uint32_t)r * 128, &tmBs, fullB0 + 8 * s, 0, row + r);
                 }
             }
         }
@@ -440,17 +596,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
                     tc_fence_after();
                     const uint32_t b_addr = smem_u32(sB) + sb_slot * (uint32_t)b_slot;
                     const int i1 = T.c_item0[c] + T.c_nitem[c];
+                    const uint64_t blo = (uint64_t)((uint32_t)T.c_half[c] * 128 >> 4);   // low parts after the high parts
+                    const uint64_t alo = (uint64_t)((uint32_t)a_bytes >> 4);
                     for (int it = T.c_item0[c]; it < i1; ++it) {
                         const uint64_t bd = desc_kmajor_sw128(b_addr + (uint32_t)T.item[it].crow * 128);
                         const uint64_t ad = desc_kmajor_sw128(a_addr + (uint32_t)T.item[it].shift * 128);
-                        const uint32_t idesc = idesc_f16_f32(256, T.item[it].n);
                         const uint32_t d = dbase + (uint32_t)T.item[it].tcol;
                         const uint32_t acc0 = (kb == 0 && T.item[it].first) ? 0u : 1u;
-                        if (issuer) {
-                            mma_f16_pair(d, ad, bd, idesc, acc0);
-                            mma_f16_pair(d, ad + 2, bd + 2, idesc, 1u);
-                            mma_f16_pair(d, ad + 4, bd + 4, idesc, 1u);
-                            mma_f16_pair(d, ad + 6, bd + 6, idesc, 1u);
+                        if constexpr (kF32) {
+                            const uint32_t idesc = idesc_tf32_f32(256, T.item[it].n);
+                            if (issuer) {
+#pragma unroll
+                                for (int q = 0; q < 4; ++q) {
+                                    mma_tf32_pair(d, ad + 2 * q, bd + 2 * q, idesc, q == 0 ? acc0 : 1u);
+                                    mma_tf32_pair(d, ad + 2 * q, bd + blo + 2 * q, idesc, 1u);
+                                    mma_tf32_pair(d, ad + alo + 2 * q, bd + 2 * q, idesc, 1u);
+                                }
+                            }
+                        } else {
+                            const uint32_t idesc = idesc_f16_f32(256, T.item[it].n);
+                            if (issuer) {
+                                mma_f16_pair(d, ad, bd, idesc, acc0);
+                                mma_f16_pair(d, ad + 2, bd + 2, idesc, 1u);
+                                mma_f16_pair(d, ad + 4, bd + 4, idesc, 1u);
+                                mma_f16_pair(d, ad + 6, bd + 6, idesc, 1u);
+                            }
                         }
                         __syncwarp();
                     }
@@ -502,7 +672,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
             const int Jx = F - Jy * HX;
             const bool pos_ok = Jx < nJx && Jy < nJy;
             const int ph0 = T.g_phase0[g], ph1 = ph0 + T.g_nphase[g];
-            __half *yimg = y + (long long)n * M * plane;
+            E *yimg = y + (long long)n * M * plane;
             int piece = 0;   // (phase, 32-channel chunk) pieces, dealt alternately to the two warps of a quarter
             for (int ph = ph0; ph < ph1;) {
                 const int rz = T.phase_r[ph][0], ry = T.phase_r[ph][1], rx = T.phase_r[ph][2];
@@ -513,7 +683,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
                 const bool pair = pair_x && ph + 1 < ph1 && (rx & 1) == 0 && T.phase_r[ph + 1][0] == rz &&
                                   T.phase_r[ph + 1][1] == ry && T.phase_r[ph + 1][2] == rx + 1;
                 const uint32_t col0 = dbase + (uint32_t)((ph - ph0) * Np);
-                __half *base = yimg + ((long long)oz * outy + oy) * outx + ox;
+                E *base = yimg + ((long long)oz * outy + oy) * outx + ox;
                 for (int m0 = 0; m0 < Np; m0 += 32, ++piece) {
                     if ((piece & 1) != eh) continue;
                     uint32_t v0[16], v1[16], w0[16], w1[16];
@@ -527,20 +697,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
                     tmem_ld_wait();
                     if (!valid) continue;
                     const int mc0 = min(16, M - m0), mc1 = min(16, M - m0 - 16);
-                    __half *dst = base + (long long)m0 * plane;
+                    E *dst = base + (long long)m0 * plane;
                     float bb[32];
                     if (bias_vec && m0 + 32 <= M) {
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const uint4 h = __ldg(reinterpret_cast<const uint4 *>(bias + m0) + j);
-                            const __half2 *h2 = reinterpret_cast<const __half2 *>(&h);
-#pragma unroll
-                            for (int q = 0; q < 4; ++q) {
-                                const float2 f = __half22float2(h2[q]);
-                                bb[8 * j + 2 * q] = f.x;
-                                bb[8 * j + 2 * q + 1] = f.y;
-                            }
-                        }
+                        ld_bias32(bias + m0, bb);
                     } else if (!has_bias) {
 #pragma unroll
                         for (int j = 0; j < 32; ++j) bb[j] = 0.f;
@@ -553,28 +713,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
 #pragma unroll
                         for (int j = 0; j < 16; ++j)
                             if (j < mc0)
-                                *reinterpret_cast<__half2 *>(dst + j * plane) =
-                                    __floats2half2_rn(act_f<ACT>(__uint_as_float(v0[j]) + bb[j]),
-                                                      act_f<ACT>(__uint_as_float(w0[j]) + bb[j]));
+                                st_pair(dst + j * plane, act_f<ACT>(__uint_as_float(v0[j]) + bb[j]),
+                                        act_f<ACT>(__uint_as_float(w0[j]) + bb[j]));
                         if (two) {
-                            __half *d1 = dst + 16 * plane;
+                            E *d1 = dst + 16 * plane;
 #pragma unroll
                             for (int j = 0; j < 16; ++j)
                                 if (j < mc1)
-                                    *reinterpret_cast<__half2 *>(d1 + j * plane) =
-                                        __floats2half2_rn(act_f<ACT>(__uint_as_float(v1[j]) + bb[16 + j]),
-                                                          act_f<ACT>(__uint_as_float(w1[j]) + bb[16 + j]));
+                                    st_pair(d1 + j * plane, act_f<ACT>(__uint_as_float(v1[j]) + bb[16 + j]),
+                                            act_f<ACT>(__uint_as_float(w1[j]) + bb[16 + j]));
                         }
                     } else {
 #pragma unroll
                         for (int j = 0; j < 16; ++j)
-                            if (j < mc0) dst[j * plane] = __float2half_rn(act_f<ACT>(__uint_as_float(v0[j]) + bb[j]));
+                            if (j < mc0) st_one(dst + j * plane, act_f<ACT>(__uint_as_float(v0[j]) + bb[j]));
                         if (two) {
-                            __half *d1 = dst + 16 * plane;
+                            E *d1 = dst + 16 * plane;
 #pragma unroll
                             for (int j = 0; j < 16; ++j)
-                                if (j < mc1)
-                                    d1[j * plane] = __float2half_rn(act_f<ACT>(__uint_as_float(v1[j]) + bb[16 + j]));
+                                if (j < mc1) st_one(d1 + j * plane, act_f<ACT>(__uint_as_float(v1[j]) + bb[16 + j]));
                         }
                     }
                 }
@@ -605,8 +762,10 @@ size_t pair_smem_bytes(const PairTables &T) {
 int round_up(int v, int m) { return (v + m - 1) / m * m; }
 
 bool build_pair_tables(const Plan &p, PairTables &T) {
-    if (p.dtype != CT_F16 || p.G != 1 || !p.tabled || p.layout != CT_NCHW) return false;
-    if (p.C < 1 || p.C % 8 != 0 || p.M < 1 || p.M > 256 || p.N < 1 || p.N > 65535) return false;
+    if ((p.dtype != CT_F16 && p.dtype != CT_F32) || p.G != 1 || !p.tabled || p.layout != CT_NCHW) return false;
+    // rows of the channels-last copy must be 16-byte multiples for TMA
+    if (p.C < 1 || p.C % (p.dtype == CT_F16 ? 8 : 4) != 0 || p.M < 1 || p.M > 256 || p.N < 1 || p.N > 65535)
+        return false;
     for (int a = 0; a < 3; ++a)
         if (p.in[a] < 1 || p.in[a] > (1 << 24) || p.out[a] > (1 << 24)) return false;
     if (p.in[0] * p.in[1] * p.in[2] >= (1LL << 31)) return false;
@@ -614,7 +773,10 @@ bool build_pair_tables(const Plan &p, PairTables &T) {
     T.C = (int32_t)p.C;
     T.M = (int32_t)p.M;
     T.Np = (int32_t)((p.M + 15) / 16 * 16);
-    T.KB = (int32_t)ceil_div(p.C, 64);
+    T.f32 = p.dtype == CT_F32;
+    T.parts = T.f32 ? 2 : 1;
+    T.cpb = T.f32 ? 32 : 64;
+    T.KB = (int32_t)ceil_div(p.C, T.cpb);
     for (int a = 0; a < 3; ++a) {
         T.in[a] = (int32_t)p.in[a];
         T.out[a] = (int32_t)p.out[a];
@@ -697,7 +859,7 @@ bool build_pair_tables(const Plan &p, PairTables &T) {
     T.chunk_rows = round_up((slice + T.n_chunks - 1) / T.n_chunks, 8);
     T.slice_rows = T.chunk_rows * T.n_chunks;
     T.a_bytes = T.n_slices * T.slice_rows * 128;
-    T.a_stride = round_up(T.a_bytes, 1024);
+    T.a_stride = round_up(T.parts * T.a_bytes, 1024);   // all parts of one stage
     const long long plane_pos = (long long)T.nJ[1] * HX;
     T.PU = (int32_t)ceil_div(plane_pos, 256);
     if ((long long)T.N * HZ * HY * HX + T.slice_rows + 256 >= (1LL << 31)) return false;
@@ -712,8 +874,8 @@ bool build_pair_tables(const Plan &p, PairTables &T) {
     const int fixed = 1024 + ((T.Np + 31) & ~31) * 4 + (2 * 4 + 2 * 12 + 5) * 8 + 16;
     T.SA = (kPSmemBudget - fixed - 3LL * T.a_stride) / 2 >= 128 * 128 ? 3 : 2;
     const long long b_room = (kPSmemBudget - fixed - (long long)T.SA * T.a_stride) / 2;   // bytes of one chunk
-    const int ch_max = (int)std::min<long long>(256, b_room / 128 / 8 * 8);                // rows per rank
-    if (ch_max < 128) return false;
+    const int ch_max = (int)std::min<long long>(256 / T.parts, b_room / 128 / T.parts / 8 * 8);   // rows per rank and part
+    if (ch_max < 128 / T.parts) return false;
     // items per group: (phase, tap) pairs grouped by input offset, offsets
     // shared by more phases first, adjacent phases merged into one wide MMA;
     // then consecutive items gathered into chunks of at most ch_max rows per rank
@@ -769,8 +931,8 @@ bool build_pair_tables(const Plan &p, PairTables &T) {
         }
         T.g_nitem[g] = (int16_t)(ni - T.g_item0[g]);
         T.g_brow[g] = rows_total;
-        T.g_rows_kb[g] = brow;
-        rows_total += brow * T.KB;
+        T.g_rows_kb[g] = brow * T.parts;
+        rows_total += brow * T.parts * T.KB;
         // chunks
         T.g_chunk0[g] = (int16_t)nc;
         int row0 = 0;
@@ -786,7 +948,7 @@ bool build_pair_tables(const Plan &p, PairTables &T) {
             T.c_nitem[nc] = (int16_t)(jt - it);
             T.c_row0[nc] = row0;
             T.c_half[nc] = half;
-            row0 += 2 * half;
+            row0 += 2 * T.parts * half;
             ++nc;
             it = jt;
         }
@@ -796,13 +958,13 @@ bool build_pair_tables(const Plan &p, PairTables &T) {
     T.total_rows = rows_total;
     // weight loads: a CTA's half of a chunk is contiguous, loaded in boxes of
     // BR rows and the remainder in boxes of BRs rows
-    int hmax = 0;
-    for (int c = 0; c < nc; ++c) hmax = std::max(hmax, (int)T.c_half[c]);
+    int hmax = 0;   // rows per rank of the largest chunk (all parts)
+    for (int c = 0; c < nc; ++c) hmax = std::max(hmax, T.parts * (int)T.c_half[c]);
     int br = 256;
     while (br > hmax) br /= 2;
     int brs = br;
     for (int c = 0; c < nc; ++c)
-        while ((T.c_half[c] % br) % brs) brs /= 2;
+        while (((T.parts * T.c_half[c]) % br) % brs) brs /= 2;
     if (br < 8 || brs < 8) return false;
     T.BR = br;
     T.BRs = brs;
@@ -838,13 +1000,13 @@ int resident_pairs(K kernel, int smem) {
 // share an SM (two pairs waiting on each other's TMEM could never proceed).
 size_t pair_launch_smem(const PairTables &T) { return std::max<size_t>(pair_smem_bytes(T), 120 * 1024); }
 
-template <int ACT>
+template <int ACT, typename E>
 ct_status launch_pair(const PairTables &T, const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmBs,
                       const void *bias, void *y, cudaStream_t st) {
     static std::atomic<int> attr_set[64];
-    if (!allow_smem(dense_pair_kernel<ACT>, attr_set, kPSmemBudget)) return CT_ERR_DEVICE;
+    if (!allow_smem(dense_pair_kernel<ACT, E>, attr_set, kPSmemBudget)) return CT_ERR_DEVICE;
     const size_t smem = pair_launch_smem(T);
-    int pairs = resident_pairs(dense_pair_kernel<ACT>, (int)smem);
+    int pairs = resident_pairs(dense_pair_kernel<ACT, E>, (int)smem);
     if (pairs > T.n_units) pairs = T.n_units;
     // programmatic dependent launch: the kernel's set-up overlaps the tail of
     // the re-layout (or the bias fill) before it; the input producer waits
@@ -858,9 +1020,9 @@ ct_status launch_pair(const PairTables &T, const CUtensorMap &tmA, const CUtenso
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const __half *b = (const __half *)bias;
-    __half *yy = (__half *)y;
-    if (cudaLaunchKernelEx(&cfg, dense_pair_kernel<ACT>, tmA, tmB, tmBs, T, b, yy) != cudaSuccess) {
+    const E *b = (const E *)bias;
+    E *yy = (E *)y;
+    if (cudaLaunchKernelEx(&cfg, dense_pair_kernel<ACT, E>, tmA, tmB, tmBs, T, b, yy) != cudaSuccess) {
         cudaGetLastError();
         return CT_ERR_DEVICE;
     }
@@ -869,11 +1031,16 @@ ct_status launch_pair(const PairTables &T, const CUtensorMap &tmA, const CUtenso
 
 }  // namespace
 
-// Automatic selection takes this kernel for one or two spatial axes.  On the
-// 3-D fp16 upsample workload (32 output channels) the halo kernel was
-// measured faster: there the epilogue's stores, not the MMAs, set the pace,
-// and the padded copy of a volume costs more than the plain re-layout.
-bool dense_pair_preferred(const Plan &p) { return p.in[0] == 1 && p.out[0] == 1 && p.k[0] == 1 && p.s[0] == 1; }
+// Automatic selection: for fp32 always (3xTF32 on the tensor cores measured
+// 5x faster than the FFMA kernel on the 1-D fp32 vocoder workload); for
+// fp16 with one or two spatial axes.  On the 3-D fp16 upsample workload (32
+// output channels) the halo kernel was measured faster: there the epilogue's
+// stores, not the MMAs, set the pace, and the padded copy of a volume costs
+// more than the plain re-layout.
+bool dense_pair_preferred(const Plan &p) {
+    if (p.dtype == CT_F32) return true;
+    return p.in[0] == 1 && p.out[0] == 1 && p.k[0] == 1 && p.s[0] == 1;
+}
 
 bool dense_pair_supports(const Plan &p) {
     PairTables *T = new PairTables();
@@ -893,15 +1060,18 @@ size_t dense_pair_packed_bytes(const Plan &p) { return (size_t)ptables(p).total_
 
 size_t dense_pair_ws_bytes(const Plan &p) {
     const PairTables &T = ptables(p);
-    return (size_t)T.N * T.HZ * T.HY * T.HX * T.C * 2;
+    return (size_t)T.parts * T.N * T.HZ * T.HY * T.HX * T.C * (T.f32 ? 4 : 2);
 }
 
 ct_status dense_pair_prepack(const Plan &p, const void *w, void *wp, cudaStream_t st) {
     const PairTables &T = ptables(p);
-    const long long total = (long long)T.total_rows * 64;
+    const long long total = (long long)T.total_rows * T.cpb;
     long long blocks = ceil_div(total, 256);
     if (blocks > 148 * 32) blocks = 148 * 32;
-    pair_prepack_kernel<<<(unsigned)blocks, 256, 0, st>>>(T, (const __half *)w, (__half *)wp);
+    if (T.f32)
+        pair_prepack_kernel<float><<<(unsigned)blocks, 256, 0, st>>>(T, (const float *)w, (float *)wp);
+    else
+        pair_prepack_kernel<__half><<<(unsigned)blocks, 256, 0, st>>>(T, (const __half *)w, (__half *)wp);
     return launch_status();
 }
 
@@ -926,34 +1096,45 @@ ct_status dense_pair_run(const Plan &p, const void *x, const void *wp, const voi
         g.ox = -T.emin[2];
         // about 8 halo stores per thread
         g.halo_blocks = (int)std::max<long long>(1, std::min<long long>(1024, ceil_div(halo_count(g).n_all * 8, 2048)));
-        if (tiles + g.halo_blocks > 0x7fffffffLL || ceil_div(T.C, kPadC) > 65535 || S >= (1LL << 31))
+        if (tiles + g.halo_blocks > 0x7fffffffLL || ceil_div(T.C, T.cpb) > 65535 || S >= (1LL << 31))
             return CT_ERR_UNSUPPORTED;
-        dim3 grid((unsigned)(tiles + g.halo_blocks), (unsigned)ceil_div(T.C, kPadC), (unsigned)T.N);
-        nchw_to_padded_kernel<<<grid, 256, 0, st>>>((const __half *)x, (__half *)ws, g);
+        dim3 grid((unsigned)(tiles + g.halo_blocks), (unsigned)ceil_div(T.C, T.cpb), (unsigned)T.N);
+        if (T.f32) {
+            float *xh = (float *)ws;
+            float *xl = xh + (size_t)T.N * T.HZ * T.HY * T.HX * T.C;
+            nchw_to_padded_f32_kernel<<<grid, 256, 0, st>>>((const float *)x, xh, xl, g);
+        } else {
+            nchw_to_padded_kernel<<<grid, 256, 0, st>>>((const __half *)x, (__half *)ws, g);
+        }
         ct_status s1 = launch_status();
         if (s1 != CT_OK) return s1;
     }
     CUtensorMap tmA, tmB, tmBs;
     {
-        const cuuint64_t dims[2] = {(cuuint64_t)T.C, (cuuint64_t)T.N * T.HZ * T.HY * T.HX};
-        const cuuint64_t strides[1] = {(cuuint64_t)T.C * 2};
-        const cuuint32_t box[2] = {64, (cuuint32_t)T.chunk_rows};
-        const cuuint32_t es[2] = {1, 1};
-        if (enc(&tmA, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, ws, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+        // (channel, padded position, part): fp32 keeps the high parts and the
+        // remainders as two planes of the workspace
+        const size_t eb = T.f32 ? 4 : 2;
+        const cuuint64_t rows = (cuuint64_t)T.N * T.HZ * T.HY * T.HX;
+        const cuuint64_t dims[3] = {(cuuint64_t)T.C, rows, (cuuint64_t)T.parts};
+        const cuuint64_t strides[2] = {(cuuint64_t)T.C * eb, (cuuint64_t)(rows * T.C * eb)};
+        const cuuint32_t box[3] = {(cuuint32_t)T.cpb, (cuuint32_t)T.chunk_rows, 1};
+        const cuuint32_t es[3] = {1, 1, 1};
+        if (enc(&tmA, T.f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, ws, dims, strides,
+                box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return CT_ERR_DEVICE;
     }
     {
-        const cuuint64_t dims[2] = {64, (cuuint64_t)T.total_rows};
+        const CUtensorMapDataType dt = T.f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+        const cuuint64_t dims[2] = {(cuuint64_t)T.cpb, (cuuint64_t)T.total_rows};
         const cuuint64_t strides[1] = {128};
         const cuuint32_t es[2] = {1, 1};
-        const cuuint32_t box[2] = {64, (cuuint32_t)T.BR};
-        const cuuint32_t box_s[2] = {64, (cuuint32_t)T.BRs};
-        if (enc(&tmB, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(wp), dims, strides, box, es,
+        const cuuint32_t box[2] = {(cuuint32_t)T.cpb, (cuuint32_t)T.BR};
+        const cuuint32_t box_s[2] = {(cuuint32_t)T.cpb, (cuuint32_t)T.BRs};
+        if (enc(&tmB, dt, 2, const_cast<void *>(wp), dims, strides, box, es,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
-            enc(&tmBs, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(wp), dims, strides, box_s, es,
+            enc(&tmBs, dt, 2, const_cast<void *>(wp), dims, strides, box_s, es,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return CT_ERR_DEVICE;
@@ -962,8 +1143,12 @@ ct_status dense_pair_run(const Plan &p, const void *x, const void *wp, const voi
         ct_status s2 = launch_dead_fill(p, bias, y, st);
         if (s2 != CT_OK) return s2;
     }
-    if (T.act == CT_ACT_RELU) return launch_pair<CT_ACT_RELU>(T, tmA, tmB, tmBs, bias, y, st);
-    return launch_pair<CT_ACT_IDENTITY>(T, tmA, tmB, tmBs, bias, y, st);
+    if (T.f32) {
+        if (T.act == CT_ACT_RELU) return launch_pair<CT_ACT_RELU, float>(T, tmA, tmB, tmBs, bias, y, st);
+        return launch_pair<CT_ACT_IDENTITY, float>(T, tmA, tmB, tmBs, bias, y, st);
+    }
+    if (T.act == CT_ACT_RELU) return launch_pair<CT_ACT_RELU, __half>(T, tmA, tmB, tmBs, bias, y, st);
+    return launch_pair<CT_ACT_IDENTITY, __half>(T, tmA, tmB, tmBs, bias, y, st);
 }
 
 }  // namespace ct

@@ -80,9 +80,9 @@ struct FillArgs {
     int32_t nhwc, has_bias, act;
 };
 
-__global__ void __launch_bounds__(256) dead_fill_kernel(const FillArgs a,
-                                                        const __half *__restrict__ bias,
-                                                        __half *__restrict__ y) {
+template <typename E>
+__global__ void __launch_bounds__(256) dead_fill_kernel(const FillArgs a, const E *__restrict__ bias,
+                                                        E *__restrict__ y) {
     const long long per_img = (long long)a.out[0] * a.out[1] * a.out[2];
     const long long total = a.N * a.M * per_img;
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
@@ -102,7 +102,7 @@ __global__ void __launch_bounds__(256) dead_fill_kernel(const FillArgs a,
         }
         const bool live = ((a.live[0] >> (o0 % a.s[0])) & 1) && ((a.live[1] >> (o1 % a.s[1])) & 1) &&
                           ((a.live[2] >> (o2 % a.s[2])) & 1);
-        if (!live) y[i] = __float2half_rn(apply_act(a.has_bias ? __half2float(bias[m]) : 0.f, a.act));
+        if (!live) y[i] = (E)apply_act(a.has_bias ? (float)bias[m] : 0.f, a.act);
     }
 }
 
@@ -141,7 +141,10 @@ ct_status launch_dead_fill(const Plan &p, const void *bias, void *y, cudaStream_
     if (total == 0) return CT_OK;
     long long blocks = ceil_div(total, 256);
     if (blocks > 148 * 64) blocks = 148 * 64;
-    dead_fill_kernel<<<(unsigned)blocks, 256, 0, st>>>(a, (const __half *)bias, (__half *)y);
+    if (p.dtype == CT_F32)
+        dead_fill_kernel<float><<<(unsigned)blocks, 256, 0, st>>>(a, (const float *)bias, (float *)y);
+    else
+        dead_fill_kernel<__half><<<(unsigned)blocks, 256, 0, st>>>(a, (const __half *)bias, (__half *)y);
     return launch_status();
 }
 

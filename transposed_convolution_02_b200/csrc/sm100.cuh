@@ -223,6 +223,27 @@ __device__ __forceinline__ void mma_f16_pair(uint32_t d_tmem, uint64_t adesc, ui
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// D[tmem] (+)= A * B^T, kind::tf32 (fp32 bit patterns read as TF32, fp32
+// accumulate), K = 8 per instruction (32 bytes of a 128-byte row).
+__device__ __forceinline__ void mma_tf32_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                              uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// 3-D tile load into this CTA's shared memory counted on the pair's barrier.
+__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap *map,
+                                                 uint32_t bar_cluster, int32_t c0, int32_t c1,
+                                                 int32_t c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+        "l"(map), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
 // Arrive on the barrier at shared offset `bar` in every CTA of `mask` once the
 // pair MMAs issued so far by this thread are done.
 __device__ __forceinline__ void mma_commit_pair_mask(uint32_t bar, uint16_t mask) {
@@ -258,6 +279,15 @@ __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t addr) {
 __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
     return (1u << 4)                    // D format: f32
            | (0u << 7) | (0u << 10)     // A, B format: f16
+           | (0u << 15) | (0u << 16)    // A, B K-major
+           | ((uint32_t)(N >> 3) << 17) // N / 8
+           | ((uint32_t)(M >> 4) << 24);// M / 16
+}
+
+// Instruction descriptor for kind::tf32: TF32 A and B (K-major), fp32 D.
+__host__ __device__ constexpr uint32_t idesc_tf32_f32(int M, int N) {
+    return (1u << 4)                    // D format: f32
+           | (2u << 7) | (2u << 10)     // A, B format: tf32
            | (0u << 15) | (0u << 16)    // A, B K-major
            | ((uint32_t)(N >> 3) << 17) // N / 8
            | ((uint32_t)(M >> 4) << 24);// M / 16
