@@ -87,13 +87,14 @@ typedef enum ct_algo {
     CT_ALGO_GROUPED = 4,   /* fp16 grouped phase kernel (mma.sync), small per-group slabs */
     CT_ALGO_DENSE_TC_PERTAP = 5, /* fp16 group-1 tcgen05 phase GEMM, one input load per tap
                                     (the general fallback of CT_ALGO_DENSE_TC) */
-    CT_ALGO_DENSE_TC_PAIR = 6    /* group-1 channels-first phase GEMM, each MMA spanning the two
-                                    SMs of a CTA pair (tcgen05 cta_group::2); fp16 (chosen
-                                    automatically for one or two spatial axes) or fp32 as
-                                    3xTF32 (TF32 high part and remainder of both operands,
-                                    three MMAs per step; chosen automatically for fp32).  The
-                                    workspace holds a zero-padded channels-last copy of X (two
-                                    planes, high parts and remainders, for fp32) */
+    CT_ALGO_DENSE_TC_PAIR = 6    /* group-1 phase GEMM, each MMA spanning the two SMs of a CTA
+                                    pair (tcgen05 cta_group::2), either layout; fp16 (chosen
+                                    automatically for channels-first with one or two spatial
+                                    axes) or fp32 as 3xTF32 (TF32 high part and remainder of
+                                    both operands, three MMAs per step; chosen automatically
+                                    for fp32).  The workspace holds a zero-padded
+                                    channels-last copy of X (two planes, high parts and
+                                    remainders, for fp32) */
 } ct_algo;
 
 /* Activation applied to every output after the bias (ClikaRT::ops::

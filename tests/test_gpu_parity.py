@@ -410,3 +410,22 @@ def test_dense_tc_pair_fp32_random_sweep():
             continue
         ran += 1
     assert ran >= 15, ran
+
+
+@pytest.mark.parametrize("dtype,case", [
+    (torch.float16, dict(x_shape=[2, 64, 11, 13], w_shape=[64, 72, 4, 4], strides=[2, 2], pads=[1, 1, 1, 1],
+                         bias=True)),
+    (torch.float16, dict(x_shape=[2, 24, 300], w_shape=[24, 40, 16], strides=[8], pads=[4, 4], bias=True)),
+    (torch.float16, dict(x_shape=[1, 16, 4, 5, 6], w_shape=[16, 24, 3, 3, 3], strides=[2, 2, 2],
+                         pads=[1, 1, 1, 1, 1, 1], output_padding=[1, 1, 1], bias=True)),
+    (torch.float32, dict(x_shape=[2, 32, 9, 10], w_shape=[32, 48, 3, 3], strides=[2, 2], dilations=[2, 2],
+                         auto_pad="SAME_UPPER", bias=True)),
+    (torch.float32, dict(x_shape=[2, 36, 200], w_shape=[36, 20, 16], strides=[8], pads=[4, 4])),
+])
+def test_dense_tc_pair_channels_last(dtype, case):
+    """Channels-last X, W ([C, k.., M]) and Y on the CTA-pair kernel: the
+    padding copy instead of the transpose, channel rows stored as 16-byte
+    pieces."""
+    full_parity(case, dtype, 83, "nhwc", algo="dense_tc_pair", expect_kernel="dense_tc_pair")
+    full_parity(dict(case, activation="relu"), dtype, 84, "nhwc", algo="dense_tc_pair",
+                expect_kernel="dense_tc_pair")

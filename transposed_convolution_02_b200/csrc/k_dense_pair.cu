@@ -62,6 +62,7 @@ struct PairTables {
     // f32: fp32 operands as a TF32 high part and its remainder (3xTF32: three
     // MMAs per step), 32 channels per 128-byte row; otherwise fp16, 64 channels
     int32_t f32, cpb, parts;            // parts: 2 (high, low) for f32, else 1
+    int32_t nhwc;                       // channels-last X, W ([C, k.., M]) and Y
     int32_t in[3], out[3], s[3], pb[3], d[3], k[3], nJ[3];   // axes z, y, x
     int32_t emin[3], HX, HY, HZ;
     int32_t n_slices, slice_rows, chunk_rows, n_chunks, a_bytes, a_stride;
@@ -137,7 +138,8 @@ __global__ void __launch_bounds__(256) pair_prepack_kernel(const __grid_constant
                 ok = ok && num % T.d[a] == 0 && ka >= 0 && ka < T.k[a];
                 kpos = kpos * T.k[a] + ka;
             }
-            if (ok) v = (float)w[((long long)ci * T.M + m) * ((long long)T.k[0] * T.k[1] * T.k[2]) + kpos];
+            const long long ksz = (long long)T.k[0] * T.k[1] * T.k[2];
+            if (ok) v = (float)(T.nhwc ? w[((long long)ci * ksz + kpos) * T.M + m] : w[((long long)ci * T.M + m) * ksz + kpos]);
         }
         if (parts == 2) v = part ? v - tf32_high(v) : tf32_high(v);
         wp[i] = (E)v;
@@ -388,6 +390,80 @@ __global__ void __launch_bounds__(256) nchw_to_padded_f32_kernel(const float *__
     }
 }
 
+// Channels-last X[n][iz][iy][ix][c] -> the same padded copy(ies): a copy of
+// 16-byte channel pieces (fp32: split into high parts and remainders), with
+// the zero halo written by the first halo_blocks blocks as above.
+template <typename E>
+__global__ void __launch_bounds__(256) nhwc_to_padded_kernel(const E *__restrict__ x, E *__restrict__ xh,
+                                                             E *__restrict__ xl, const PadGeo g) {
+    constexpr int kPer = 16 / sizeof(E);   // elements per 16-byte piece
+    const int n = blockIdx.z;
+    const int C = g.C, H = g.H, W = g.W, HY = g.HY, HX = g.HX;
+    const long long HW = (long long)H * W;
+    const long long S = g.D * HW;
+    const long long P2 = (long long)HY * HX;
+    const long long P = g.HZ * P2;
+    const int t = threadIdx.x;
+    const int cch = C / kPer;   // pieces per position
+    sm100::griddep_launch_dependents();   // the pair kernel may set up while this one runs
+    if ((int)blockIdx.x < g.halo_blocks) {
+        const HaloCount h = halo_count(g);
+        const long long work = h.n_all * cch;
+        for (long long q = (long long)blockIdx.x * blockDim.x + t; q < work; q += (long long)g.halo_blocks * blockDim.x) {
+            const long long k = q / cch;
+            const int cc = (int)(q - k * cch);
+            long long pos;
+            if (k < h.n_zt || k >= h.n_zt + h.n_zm) {
+                pos = k < h.n_zt ? k : (long long)h.zmid_end * P2 + (k - h.n_zt - h.n_zm);
+            } else {
+                const int kk = (int)(k - h.n_zt);
+                const int zq = kk / h.h2;
+                const int k2 = kk - zq * h.h2;
+                int yp, xq;
+                if (k2 < h.n_top) {
+                    yp = k2 / HX;
+                    xq = k2 - yp * HX;
+                } else if (k2 < h.n_top + h.n_mid) {
+                    const int r = (k2 - h.n_top) / h.lr, j = (k2 - h.n_top) - r * h.lr;
+                    yp = h.top + r;
+                    xq = j < h.left ? j : h.right0 + (j - h.left);
+                } else {
+                    const int k3 = k2 - h.n_top - h.n_mid;
+                    yp = h.mid_end + k3 / HX;
+                    xq = k3 - (k3 / HX) * HX;
+                }
+                pos = (long long)(h.ztop + zq) * P2 + (long long)yp * HX + xq;
+            }
+            const long long off = ((long long)n * P + pos) * C + (long long)cc * kPer;
+            *reinterpret_cast<uint4 *>(xh + off) = make_uint4(0, 0, 0, 0);
+            if (xl) *reinterpret_cast<uint4 *>(xl + off) = make_uint4(0, 0, 0, 0);
+        }
+        return;
+    }
+    const long long work = S * cch;
+    const long long stride = (long long)(gridDim.x - g.halo_blocks) * blockDim.x;
+    for (long long q = (long long)(blockIdx.x - g.halo_blocks) * blockDim.x + t; q < work; q += stride) {
+        const long long sidx = q / cch;
+        const int cc = (int)(q - sidx * cch);
+        const int iz = (int)sidx / (int)HW;   // S < 2^31
+        const int rem = (int)sidx - iz * (int)HW;
+        const int iy = rem / W, ix = rem - iy * W;
+        const int zp = iz + g.oz, yp = iy + g.oy, xq = ix + g.ox;
+        if (zp < 0 || zp >= g.HZ || yp < 0 || yp >= HY || xq < 0 || xq >= HX) continue;
+        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(x + ((long long)n * S + sidx) * C) + cc);
+        const long long off = ((long long)n * P + zp * P2 + (long long)yp * HX + xq) * C + (long long)cc * kPer;
+        if (xl) {
+            // fp32: the TF32 high parts and the remainders
+            const float4 f = *reinterpret_cast<const float4 *>(&v);
+            const float4 hi = make_float4(tf32_high(f.x), tf32_high(f.y), tf32_high(f.z), tf32_high(f.w));
+            *reinterpret_cast<float4 *>(xh + off) = hi;
+            *reinterpret_cast<float4 *>(xl + off) = make_float4(f.x - hi.x, f.y - hi.y, f.z - hi.z, f.w - hi.w);
+        } else {
+            *reinterpret_cast<uint4 *>(xh + off) = v;
+        }
+    }
+}
+
 // ---------------------------------------------------------------------------
 // A unit: image n, output slice jz, group g, pair positions [pu*256, +256) of
 // the slice; rank r of the pair owns [pu*256 + 128*r, +128).  Units are
@@ -429,6 +505,41 @@ __device__ __forceinline__ void ld_bias32(const float *b, float (&bb)[32]) {
         bb[4 * j + 1] = f.y;
         bb[4 * j + 2] = f.z;
         bb[4 * j + 3] = f.w;
+    }
+}
+
+// 16 consecutive channels of one channels-last position: 16-byte stores when
+// the row is whole and aligned, else element by element.
+template <int ACT>
+__device__ __forceinline__ void store_row16(__half *dst, const uint32_t (&v)[16], const float *b, int mc) {
+    if (mc == 16 && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+        uint4 q[2];
+        __half2 *h = reinterpret_cast<__half2 *>(q);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            h[j] = __floats2half2_rn(apply_act(__uint_as_float(v[2 * j]) + b[2 * j], ACT),
+                                     apply_act(__uint_as_float(v[2 * j + 1]) + b[2 * j + 1], ACT));
+        reinterpret_cast<uint4 *>(dst)[0] = q[0];
+        reinterpret_cast<uint4 *>(dst)[1] = q[1];
+    } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            if (j < mc) dst[j] = __float2half_rn(apply_act(__uint_as_float(v[j]) + b[j], ACT));
+    }
+}
+template <int ACT>
+__device__ __forceinline__ void store_row16(float *dst, const uint32_t (&v)[16], const float *b, int mc) {
+    if (mc == 16 && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            reinterpret_cast<float4 *>(dst)[j] = make_float4(apply_act(__uint_as_float(v[4 * j]) + b[4 * j], ACT),
+                                                             apply_act(__uint_as_float(v[4 * j + 1]) + b[4 * j + 1], ACT),
+                                                             apply_act(__uint_as_float(v[4 * j + 2]) + b[4 * j + 2], ACT),
+                                                             apply_act(__uint_as_float(v[4 * j + 3]) + b[4 * j + 3], ACT));
+    } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            if (j < mc) dst[j] = apply_act(__uint_as_float(v[j]) + b[j], ACT);
     }
 }
 
@@ -653,7 +764,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
         const int p = lane_base + lane;
         const int outz = T.out[0], outy = T.out[1], outx = T.out[2];
         const int sz = T.s[0], sy = T.s[1], sx = T.s[2], nJy = T.nJ[1], nJx = T.nJ[2];
-        const int pair_x = T.pair_x;
+        const int pair_x = T.pair_x, nhwc = T.nhwc;
         const bool has_bias = T.has_bias;
         const bool bias_vec = has_bias && (reinterpret_cast<uintptr_t>(bias) & 15) == 0;
         const long long plane = (long long)outz * outy * outx;
@@ -683,7 +794,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
                 const bool pair = pair_x && ph + 1 < ph1 && (rx & 1) == 0 && T.phase_r[ph + 1][0] == rz &&
                                   T.phase_r[ph + 1][1] == ry && T.phase_r[ph + 1][2] == rx + 1;
                 const uint32_t col0 = dbase + (uint32_t)((ph - ph0) * Np);
-                E *base = yimg + ((long long)oz * outy + oy) * outx + ox;
+                const long long opos = ((long long)oz * outy + oy) * outx + ox;
+                E *base = yimg + opos;                  // channels-first: channel stride plane
+                E *rowl = yimg + opos * M;              // channels-last: the position's channel row
                 for (int m0 = 0; m0 < Np; m0 += 32, ++piece) {
                     if ((piece & 1) != eh) continue;
                     uint32_t v0[16], v1[16], w0[16], w1[16];
@@ -708,7 +821,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
 #pragma unroll
                         for (int j = 0; j < 32; ++j) bb[j] = bias_s[m0 + j];
                     }
-                    if (pair) {
+                    if (nhwc) {
+                        // channels-last: 16 channels of a position as 16-byte pieces;
+                        // the second x phase is the next position
+                        E *dr = rowl + m0;
+                        store_row16<ACT>(dr, v0, bb, mc0);
+                        if (two) store_row16<ACT>(dr + 16, v1, bb + 16, mc1);
+                        if (pair) {
+                            store_row16<ACT>(dr + M, w0, bb, mc0);
+                            if (two) store_row16<ACT>(dr + M + 16, w1, bb + 16, mc1);
+                        }
+                    } else if (pair) {
                         // both x phases of a channel are adjacent: one half2 per channel
 #pragma unroll
                         for (int j = 0; j < 16; ++j)
@@ -762,7 +885,7 @@ size_t pair_smem_bytes(const PairTables &T) {
 int round_up(int v, int m) { return (v + m - 1) / m * m; }
 
 bool build_pair_tables(const Plan &p, PairTables &T) {
-    if ((p.dtype != CT_F16 && p.dtype != CT_F32) || p.G != 1 || !p.tabled || p.layout != CT_NCHW) return false;
+    if ((p.dtype != CT_F16 && p.dtype != CT_F32) || p.G != 1 || !p.tabled) return false;
     // rows of the channels-last copy must be 16-byte multiples for TMA
     if (p.C < 1 || p.C % (p.dtype == CT_F16 ? 8 : 4) != 0 || p.M < 1 || p.M > 256 || p.N < 1 || p.N > 65535)
         return false;
@@ -774,6 +897,7 @@ bool build_pair_tables(const Plan &p, PairTables &T) {
     T.M = (int32_t)p.M;
     T.Np = (int32_t)((p.M + 15) / 16 * 16);
     T.f32 = p.dtype == CT_F32;
+    T.nhwc = p.layout == CT_NHWC;
     T.parts = T.f32 ? 2 : 1;
     T.cpb = T.f32 ? 32 : 64;
     T.KB = (int32_t)ceil_div(p.C, T.cpb);
@@ -1032,14 +1156,16 @@ ct_status launch_pair(const PairTables &T, const CUtensorMap &tmA, const CUtenso
 }  // namespace
 
 // Automatic selection: for fp32 always (3xTF32 on the tensor cores measured
-// 5x faster than the FFMA kernel on the 1-D fp32 vocoder workload); for
-// fp16 with one or two spatial axes.  On the 3-D fp16 upsample workload (32
-// output channels) the halo kernel was measured faster: there the epilogue's
-// stores, not the MMAs, set the pace, and the padded copy of a volume costs
-// more than the plain re-layout.
+// 5x (channels-first) and 8x (channels-last) faster than the FFMA kernel on
+// the 1-D fp32 vocoder workload); for fp16 channels-first with one or two
+// spatial axes.  On the 3-D fp16 upsample workload (32 output channels) the
+// halo kernel was measured faster: there the epilogue's stores, not the
+// MMAs, set the pace, and the padded copy of a volume costs more than the
+// plain re-layout.  For fp16 channels-last the two measured the same on the
+// 2-D decoder workload, and the halo kernel needs no workspace.
 bool dense_pair_preferred(const Plan &p) {
     if (p.dtype == CT_F32) return true;
-    return p.in[0] == 1 && p.out[0] == 1 && p.k[0] == 1 && p.s[0] == 1;
+    return p.layout == CT_NCHW && p.in[0] == 1 && p.out[0] == 1 && p.k[0] == 1 && p.s[0] == 1;
 }
 
 bool dense_pair_supports(const Plan &p) {
@@ -1099,9 +1225,21 @@ ct_status dense_pair_run(const Plan &p, const void *x, const void *wp, const voi
         if (tiles + g.halo_blocks > 0x7fffffffLL || ceil_div(T.C, T.cpb) > 65535 || S >= (1LL << 31))
             return CT_ERR_UNSUPPORTED;
         dim3 grid((unsigned)(tiles + g.halo_blocks), (unsigned)ceil_div(T.C, T.cpb), (unsigned)T.N);
-        if (T.f32) {
+        const size_t plane_elems = (size_t)T.N * T.HZ * T.HY * T.HX * T.C;
+        if (T.nhwc) {
+            // channels-last X: a padding copy of 16-byte pieces, about 8 per thread
+            const long long pieces = (long long)T.C / (T.f32 ? 4 : 8);
+            g.halo_blocks = (int)std::max<long long>(1, std::min<long long>(1024, ceil_div(halo_count(g).n_all * pieces, 2048)));
+            const long long copy_blocks = std::max<long long>(1, std::min<long long>(8192, ceil_div(S * pieces, 2048)));
+            dim3 gridc((unsigned)(g.halo_blocks + copy_blocks), 1, (unsigned)T.N);
+            if (T.f32)
+                nhwc_to_padded_kernel<float><<<gridc, 256, 0, st>>>((const float *)x, (float *)ws,
+                                                                    (float *)ws + plane_elems, g);
+            else
+                nhwc_to_padded_kernel<__half><<<gridc, 256, 0, st>>>((const __half *)x, (__half *)ws, nullptr, g);
+        } else if (T.f32) {
             float *xh = (float *)ws;
-            float *xl = xh + (size_t)T.N * T.HZ * T.HY * T.HX * T.C;
+            float *xl = xh + plane_elems;
             nchw_to_padded_f32_kernel<<<grid, 256, 0, st>>>((const float *)x, xh, xl, g);
         } else {
             nchw_to_padded_kernel<<<grid, 256, 0, st>>>((const __half *)x, (__half *)ws, g);
