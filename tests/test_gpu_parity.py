@@ -429,3 +429,23 @@ def test_dense_tc_pair_channels_last(dtype, case):
     full_parity(case, dtype, 83, "nhwc", algo="dense_tc_pair", expect_kernel="dense_tc_pair")
     full_parity(dict(case, activation="relu"), dtype, 84, "nhwc", algo="dense_tc_pair",
                 expect_kernel="dense_tc_pair")
+
+
+@pytest.mark.parametrize("dtype,layout,case", [
+    # 300 output channels: two tiles of 160, the second partly beyond M
+    (torch.float16, "nchw", dict(x_shape=[2, 64, 9, 11], w_shape=[64, 300, 4, 4], strides=[2, 2],
+                                 pads=[1, 1, 1, 1], bias=True)),
+    # 3-D with 320 output channels (no tuned fp16 kernel takes more than 256)
+    (torch.float16, "nchw", dict(x_shape=[1, 32, 4, 5, 6], w_shape=[32, 320, 3, 3, 3], strides=[2, 2, 2],
+                                 pads=[1, 1, 1, 1, 1, 1], output_padding=[1, 1, 1], bias=True)),
+    (torch.float16, "nhwc", dict(x_shape=[2, 32, 7, 9], w_shape=[32, 272, 3, 3], strides=[2, 2],
+                                 pads=[1, 1, 1, 1], bias=True)),
+    (torch.float32, "nchw", dict(x_shape=[2, 36, 100], w_shape=[36, 512, 16], strides=[8], pads=[4, 4],
+                                 bias=True)),
+])
+def test_dense_tc_pair_channel_tiles(dtype, layout, case):
+    """More than 256 output channels: the pair kernel walks output-channel
+    tiles of at most 256 (one MMA's N); automatic selection takes it."""
+    full_parity(case, dtype, 85, layout, expect_kernel="dense_tc_pair")
+    full_parity(dict(case, activation="relu"), dtype, 86, layout, algo="dense_tc_pair",
+                expect_kernel="dense_tc_pair")

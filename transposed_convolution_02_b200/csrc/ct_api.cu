@@ -160,6 +160,10 @@ void choose(Plan *p) {
         p->algo = CT_ALGO_GROUPED;
     } else if ((want == CT_ALGO_AUTO || want == CT_ALGO_FP32_GEMM) && fp32_gemm_supports(*p)) {
         p->algo = CT_ALGO_FP32_GEMM;
+    } else if (want == CT_ALGO_AUTO && dense_pair_supports(*p)) {
+        // dense shapes the tuned choices above do not take (more than 256
+        // output channels, for one)
+        p->algo = CT_ALGO_DENSE_TC_PAIR;
     } else if (want != CT_ALGO_AUTO) {
         p->algo = -1;
     }

@@ -63,6 +63,9 @@ struct PairTables {
     // MMAs per step), 32 channels per 128-byte row; otherwise fp16, 64 channels
     int32_t f32, cpb, parts;            // parts: 2 (high, low) for f32, else 1
     int32_t nhwc;                       // channels-last X, W ([C, k.., M]) and Y
+    // output channels in n_mt tiles of Mt (= Np) channels; every tile has the
+    // same groups and items, and its own total_rows of packed weights
+    int32_t Mt, n_mt, BL;               // BL: bias entries kept in shared memory
     int32_t in[3], out[3], s[3], pb[3], d[3], k[3], nJ[3];   // axes z, y, x
     int32_t emin[3], HX, HY, HZ;
     int32_t n_slices, slice_rows, chunk_rows, n_chunks, a_bytes, a_stride;
@@ -101,11 +104,13 @@ template <typename E>
 __global__ void __launch_bounds__(256) pair_prepack_kernel(const __grid_constant__ PairTables T,
                                                            const E *__restrict__ w, E *__restrict__ wp) {
     const int cpb = T.cpb, parts = T.parts;
-    const long long total = (long long)T.total_rows * cpb;
+    const long long total = (long long)T.n_mt * T.total_rows * cpb;
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
          i += (long long)gridDim.x * blockDim.x) {
         const int cc = (int)(i % cpb);
-        const int row = (int)(i / cpb);
+        const int row_all = (int)(i / cpb);
+        const int mt = row_all / T.total_rows;   // output-channel tile
+        const int row = row_all - mt * T.total_rows;
         int g = 0;
         while (g + 1 < T.n_groups && row >= T.g_brow[g + 1]) ++g;
         const int rg = row - T.g_brow[g];
@@ -126,7 +131,7 @@ __global__ void __launch_bounds__(256) pair_prepack_kernel(const __grid_constant
         const PItem &I = T.item[it];
         const int rr = rank * (I.n / 2) + (r4 - I.crow);
         const int ph = I.phase0 + rr / T.Np;
-        const int m = rr % T.Np;
+        const int m = mt * T.Mt + rr % T.Np;   // output channel
         const int ci = kb * cpb + cc;
         float v = 0.f;
         if (ci < T.C && m < T.M) {
@@ -569,7 +574,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
     uint8_t *sA = smem;
     uint8_t *sB = sA + (size_t)SA * a_stride;
     float *bias_s = reinterpret_cast<float *>(sB + (size_t)SB * b_slot);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(bias_s + ((Np + 31) & ~31));   // 128-byte multiple: aligned
+    uint64_t *bars = reinterpret_cast<uint64_t *>(bias_s + T.BL);   // BL is a multiple of 32: aligned
     const uint32_t fullA = smem_u32(bars), emptyA = smem_u32(bars + SA);
     const uint32_t fullB = smem_u32(bars + 2 * SA), emptyB = smem_u32(bars + 2 * SA + SB);
     const uint32_t tfull = smem_u32(bars + 2 * SA + 2 * SB);
@@ -596,7 +601,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
         prefetch_tmap(&tmB);
         prefetch_tmap(&tmBs);
     }
-    for (int m = threadIdx.x; m < ((Np + 31) & ~31); m += kPThreads)
+    for (int m = threadIdx.x; m < T.BL; m += kPThreads)
         bias_s[m] = (T.has_bias && m < M) ? (float)bias[m] : 0.f;
     if (warp == 1) {
         tmem_alloc_pair(smem_u32(tmem_slot), 512);
@@ -619,7 +624,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
         int ia = 0;
         bool ok = true;
         for (int u = cid; u < n_units && ok; u += ncl) {
-            int t = u / ng;
+            int t = u / ng / T.n_mt;   // the channel tile does not change the input
             const int pu = t % PU;
             t /= PU;
             const int jz = t % nJz, n = t / nJz;
@@ -654,7 +659,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
             const int g = u % ng;
             const int c0 = T.g_chunk0[g], c1 = c0 + T.g_nchunk[g];
             for (int kb = 0; kb < KB && ok; ++kb) {
-                const int rowbase = T.g_brow[g] + kb * T.g_rows_kb[g];
+                const int rowbase = ((u / ng) % T.n_mt) * T.total_rows + T.g_brow[g] + kb * T.g_rows_kb[g];
                 for (int c = c0; c < c1; ++c, ++ib) {
                     if ((ib & 1) != me) continue;
                     const int s = ib % SB;
@@ -771,7 +776,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
         int local = 0;
         for (int u = cid; u < n_units; u += ncl, ++local) {
             const int g = u % ng;
-            const int t = u / ng;
+            const int mt = (u / ng) % T.n_mt;
+            const int t = u / ng / T.n_mt;
             const int pu = t % PU;
             const int jz = (t / PU) % nJz, n = (t / PU) / nJz;
             const int buf = local & 1, use = local >> 1;
@@ -784,6 +790,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
             const bool pos_ok = Jx < nJx && Jy < nJy;
             const int ph0 = T.g_phase0[g], ph1 = ph0 + T.g_nphase[g];
             E *yimg = y + (long long)n * M * plane;
+            const int cb = mt * T.Mt;                 // first output channel of this tile
+            const int Mrem = min(T.Mt, M - cb);       // its channels that exist
             int piece = 0;   // (phase, 32-channel chunk) pieces, dealt alternately to the two warps of a quarter
             for (int ph = ph0; ph < ph1;) {
                 const int rz = T.phase_r[ph][0], ry = T.phase_r[ph][1], rx = T.phase_r[ph][2];
@@ -809,22 +817,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
                     }
                     tmem_ld_wait();
                     if (!valid) continue;
-                    const int mc0 = min(16, M - m0), mc1 = min(16, M - m0 - 16);
-                    E *dst = base + (long long)m0 * plane;
+                    const int mc0 = min(16, Mrem - m0), mc1 = min(16, Mrem - m0 - 16);
+                    E *dst = base + (long long)(cb + m0) * plane;
                     float bb[32];
-                    if (bias_vec && m0 + 32 <= M) {
-                        ld_bias32(bias + m0, bb);
+                    if (bias_vec && m0 + 32 <= Mrem) {
+                        ld_bias32(bias + cb + m0, bb);
                     } else if (!has_bias) {
 #pragma unroll
                         for (int j = 0; j < 32; ++j) bb[j] = 0.f;
                     } else {   // the last, partial chunk of channels, or an unaligned bias
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) bb[j] = bias_s[m0 + j];
+                        for (int j = 0; j < 32; ++j) bb[j] = bias_s[cb + m0 + j];
                     }
                     if (nhwc) {
                         // channels-last: 16 channels of a position as 16-byte pieces;
                         // the second x phase is the next position
-                        E *dr = rowl + m0;
+                        E *dr = rowl + cb + m0;
                         store_row16<ACT>(dr, v0, bb, mc0);
                         if (two) store_row16<ACT>(dr + 16, v1, bb + 16, mc1);
                         if (pair) {
@@ -875,7 +883,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
 }
 
 size_t pair_smem_bytes(const PairTables &T) {
-    return 1024 + (size_t)T.SA * T.a_stride + (size_t)T.SB * T.b_slot + (size_t)((T.Np + 31) & ~31) * 4 +
+    return 1024 + (size_t)T.SA * T.a_stride + (size_t)T.SB * T.b_slot + (size_t)T.BL * 4 +
            (size_t)(2 * T.SA + 2 * T.SB + 5) * 8 + 16;
 }
 
@@ -887,7 +895,7 @@ int round_up(int v, int m) { return (v + m - 1) / m * m; }
 bool build_pair_tables(const Plan &p, PairTables &T) {
     if ((p.dtype != CT_F16 && p.dtype != CT_F32) || p.G != 1 || !p.tabled) return false;
     // rows of the channels-last copy must be 16-byte multiples for TMA
-    if (p.C < 1 || p.C % (p.dtype == CT_F16 ? 8 : 4) != 0 || p.M < 1 || p.M > 256 || p.N < 1 || p.N > 65535)
+    if (p.C < 1 || p.C % (p.dtype == CT_F16 ? 8 : 4) != 0 || p.M < 1 || p.M > 16384 || p.N < 1 || p.N > 65535)
         return false;
     for (int a = 0; a < 3; ++a)
         if (p.in[a] < 1 || p.in[a] > (1 << 24) || p.out[a] > (1 << 24)) return false;
@@ -895,7 +903,11 @@ bool build_pair_tables(const Plan &p, PairTables &T) {
     T.N = (int32_t)p.N;
     T.C = (int32_t)p.C;
     T.M = (int32_t)p.M;
-    T.Np = (int32_t)((p.M + 15) / 16 * 16);
+    // output channels in tiles of at most 256 (one MMA's N), as even as 16 allows
+    T.n_mt = (int32_t)ceil_div(p.M, 256);
+    T.Mt = (int32_t)((ceil_div(p.M, T.n_mt) + 15) / 16 * 16);
+    T.Np = T.Mt;
+    T.BL = (T.n_mt * T.Mt + 31) / 32 * 32;
     T.f32 = p.dtype == CT_F32;
     T.nhwc = p.layout == CT_NHWC;
     T.parts = T.f32 ? 2 : 1;
@@ -987,7 +999,7 @@ bool build_pair_tables(const Plan &p, PairTables &T) {
     const long long plane_pos = (long long)T.nJ[1] * HX;
     T.PU = (int32_t)ceil_div(plane_pos, 256);
     if ((long long)T.N * HZ * HY * HX + T.slice_rows + 256 >= (1LL << 31)) return false;
-    const long long units = (long long)T.N * T.nJ[0] * T.PU * ng;
+    const long long units = (long long)T.N * T.nJ[0] * T.PU * ng * T.n_mt;
     if (units > (1LL << 30)) return false;
     T.n_units = (int32_t)units;
     // shared memory: three input stages (two when they do not fit) and at
@@ -995,7 +1007,7 @@ bool build_pair_tables(const Plan &p, PairTables &T) {
     // 2-D decoder workload, three 34 KB input stages with three 32 KB chunk
     // slots beat two input stages with 64 KB chunks: the loads, not the
     // MMAs, set the pace there.
-    const int fixed = 1024 + ((T.Np + 31) & ~31) * 4 + (2 * 4 + 2 * 12 + 5) * 8 + 16;
+    const int fixed = 1024 + T.BL * 4 + (2 * 4 + 2 * 12 + 5) * 8 + 16;
     T.SA = (kPSmemBudget - fixed - 3LL * T.a_stride) / 2 >= 128 * 128 ? 3 : 2;
     const long long b_room = (kPSmemBudget - fixed - (long long)T.SA * T.a_stride) / 2;   // bytes of one chunk
     const int ch_max = (int)std::min<long long>(256 / T.parts, b_room / 128 / T.parts / 8 * 8);   // rows per rank and part
@@ -1080,6 +1092,7 @@ bool build_pair_tables(const Plan &p, PairTables &T) {
     }
     T.n_items = ni;
     T.total_rows = rows_total;
+    if ((long long)T.n_mt * rows_total >= (1LL << 30)) return false;
     // weight loads: a CTA's half of a chunk is contiguous, loaded in boxes of
     // BR rows and the remainder in boxes of BRs rows
     int hmax = 0;   // rows per rank of the largest chunk (all parts)
@@ -1182,7 +1195,7 @@ void dense_pair_setup(Plan &p) {
     p.launches = 2 + (T.dead ? 1 : 0);
 }
 
-size_t dense_pair_packed_bytes(const Plan &p) { return (size_t)ptables(p).total_rows * 128; }
+size_t dense_pair_packed_bytes(const Plan &p) { return (size_t)ptables(p).n_mt * ptables(p).total_rows * 128; }
 
 size_t dense_pair_ws_bytes(const Plan &p) {
     const PairTables &T = ptables(p);
@@ -1191,7 +1204,7 @@ size_t dense_pair_ws_bytes(const Plan &p) {
 
 ct_status dense_pair_prepack(const Plan &p, const void *w, void *wp, cudaStream_t st) {
     const PairTables &T = ptables(p);
-    const long long total = (long long)T.total_rows * T.cpb;
+    const long long total = (long long)T.n_mt * T.total_rows * T.cpb;
     long long blocks = ceil_div(total, 256);
     if (blocks > 148 * 32) blocks = 148 * 32;
     if (T.f32)
@@ -1264,7 +1277,7 @@ ct_status dense_pair_run(const Plan &p, const void *x, const void *wp, const voi
     }
     {
         const CUtensorMapDataType dt = T.f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-        const cuuint64_t dims[2] = {(cuuint64_t)T.cpb, (cuuint64_t)T.total_rows};
+        const cuuint64_t dims[2] = {(cuuint64_t)T.cpb, (cuuint64_t)T.n_mt * T.total_rows};
         const cuuint64_t strides[1] = {128};
         const cuuint32_t es[2] = {1, 1};
         const cuuint32_t box[2] = {(cuuint32_t)T.cpb, (cuuint32_t)T.BR};
