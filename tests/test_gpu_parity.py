@@ -449,3 +449,18 @@ def test_dense_tc_pair_channel_tiles(dtype, layout, case):
     full_parity(case, dtype, 85, layout, expect_kernel="dense_tc_pair")
     full_parity(dict(case, activation="relu"), dtype, 86, layout, algo="dense_tc_pair",
                 expect_kernel="dense_tc_pair")
+
+
+@pytest.mark.parametrize("dtype,case", [
+    # (sizes above the 10 MFLOP below which the generic kernel is chosen)
+    (torch.float16, dict(x_shape=[4, 3, 40, 48], w_shape=[3, 64, 4, 4], strides=[2, 2], pads=[1, 1, 1, 1],
+                         bias=True)),
+    (torch.float16, dict(x_shape=[2, 12, 8, 10, 12], w_shape=[12, 16, 3, 3, 3], strides=[2, 2, 2],
+                         pads=[1, 1, 1, 1, 1, 1], bias=True)),
+    (torch.float32, dict(x_shape=[4, 5, 2000], w_shape=[5, 24, 8], strides=[4], pads=[2, 2], bias=True)),
+])
+def test_dense_tc_pair_channels_padded(dtype, case):
+    """Input channels that do not fill a 16-byte row (C = 3, 12, 5): the
+    channels-first re-layout pads them with zeros; automatic selection takes
+    the pair kernel instead of the generic one."""
+    full_parity(case, dtype, 87, "nchw", expect_kernel="dense_tc_pair")

@@ -66,6 +66,7 @@ struct PairTables {
     // output channels in n_mt tiles of Mt (= Np) channels; every tile has the
     // same groups and items, and its own total_rows of packed weights
     int32_t Mt, n_mt, BL;               // BL: bias entries kept in shared memory
+    int32_t Cd;                         // channels of a padded position: C rounded up to a 16-byte row
     int32_t in[3], out[3], s[3], pb[3], d[3], k[3], nJ[3];   // axes z, y, x
     int32_t emin[3], HX, HY, HZ;
     int32_t n_slices, slice_rows, chunk_rows, n_chunks, a_bytes, a_stride;
@@ -163,6 +164,7 @@ constexpr int kPadC = 64, kPadS = 128;
 
 struct PadGeo {
     int C, D, H, W;      // input extents
+    int Cd;              // channels of a padded position (C rounded up to a 16-byte row)
     int HZ, HY, HX;      // padded extents
     int oz, oy, ox;      // padded origin: zp = iz + oz, ...
     int halo_blocks;     // blocks x = 0..halo_blocks-1 write the zero halo
@@ -197,7 +199,7 @@ __host__ __device__ inline HaloCount halo_count(const PadGeo &g) {
 __global__ void __launch_bounds__(256) nchw_to_padded_kernel(const __half *__restrict__ x,
                                                              __half *__restrict__ xp, const PadGeo g) {
     const int n = blockIdx.z;
-    const int C = g.C, H = g.H, W = g.W, HY = g.HY, HX = g.HX;
+    const int C = g.C, Cd = g.Cd, H = g.H, W = g.W, HY = g.HY, HX = g.HX;
     const long long HW = (long long)H * W;
     const long long S = g.D * HW;
     const long long P2 = (long long)HY * HX;
@@ -207,9 +209,9 @@ __global__ void __launch_bounds__(256) nchw_to_padded_kernel(const __half *__res
     if ((int)blockIdx.x < g.halo_blocks) {
         // zero halo of image n, channels [c0, c0 + 64), spread over the halo blocks
         const int c0 = blockIdx.y * kPadC;
-        const int c8 = (min(kPadC, C - c0)) >> 3;
+        const int c8 = (min(kPadC, Cd - c0)) >> 3;
         const HaloCount h = halo_count(g);
-        __half *img = xp + (long long)n * P * C + c0;
+        __half *img = xp + (long long)n * P * Cd + c0;
         const long long work = h.n_all * c8;
         for (long long q = (long long)blockIdx.x * blockDim.x + t; q < work; q += (long long)g.halo_blocks * blockDim.x) {
             const long long k = q / c8;
@@ -236,7 +238,7 @@ __global__ void __launch_bounds__(256) nchw_to_padded_kernel(const __half *__res
                 }
                 pos = (long long)(h.ztop + zq) * P2 + (long long)yp * HX + xq;
             }
-            *reinterpret_cast<uint4 *>(img + pos * C + cc * 8) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4 *>(img + pos * Cd + cc * 8) = make_uint4(0, 0, 0, 0);
         }
         return;
     }
@@ -275,7 +277,7 @@ __global__ void __launch_bounds__(256) nchw_to_padded_kernel(const __half *__res
         for (int r = 0; r < 4; ++r) {
             const int sp = sl + 32 * r;
             const long long s = s0 + sp;
-            if (s >= S || c >= C) continue;
+            if (s >= S || c >= Cd) continue;   // channels C..Cd of the row are zeros
             const int iz = (int)s / (int)HW;                      // S < 2^31
             const int rem = (int)s - iz * (int)HW;
             const int iy = rem / W, ix = rem - iy * W;
@@ -285,7 +287,7 @@ __global__ void __launch_bounds__(256) nchw_to_padded_kernel(const __half *__res
             const int col = (((sp >> 3) ^ cv) << 3) | (sp & 7);
 #pragma unroll
             for (int j = 0; j < 8; ++j) v[j] = tile[cv * 8 + j][col];
-            *reinterpret_cast<uint4 *>(xp + ((long long)n * P + zp * P2 + (long long)yp * HX + xq) * C + c) =
+            *reinterpret_cast<uint4 *>(xp + ((long long)n * P + zp * P2 + (long long)yp * HX + xq) * Cd + c) =
                 *reinterpret_cast<const uint4 *>(v);
         }
     }
@@ -301,7 +303,7 @@ __global__ void __launch_bounds__(256) nchw_to_padded_f32_kernel(const float *__
                                                                  float *__restrict__ xh, float *__restrict__ xl,
                                                                  const PadGeo g) {
     const int n = blockIdx.z;
-    const int C = g.C, H = g.H, W = g.W, HY = g.HY, HX = g.HX;
+    const int C = g.C, Cd = g.Cd, H = g.H, W = g.W, HY = g.HY, HX = g.HX;
     const long long HW = (long long)H * W;
     const long long S = g.D * HW;
     const long long P2 = (long long)HY * HX;
@@ -310,7 +312,7 @@ __global__ void __launch_bounds__(256) nchw_to_padded_f32_kernel(const float *__
     sm100::griddep_launch_dependents();   // the pair kernel may set up while this one runs
     if ((int)blockIdx.x < g.halo_blocks) {
         const int c0 = blockIdx.y * kPadC32;
-        const int c4 = (min(kPadC32, C - c0)) >> 2;
+        const int c4 = (min(kPadC32, Cd - c0)) >> 2;
         const HaloCount h = halo_count(g);
         const long long work = h.n_all * c4;
         for (long long q = (long long)blockIdx.x * blockDim.x + t; q < work; q += (long long)g.halo_blocks * blockDim.x) {
@@ -338,7 +340,7 @@ __global__ void __launch_bounds__(256) nchw_to_padded_f32_kernel(const float *__
                 }
                 pos = (long long)(h.ztop + zq) * P2 + (long long)yp * HX + xq;
             }
-            const long long off = ((long long)n * P + pos) * C + c0 + cc * 4;
+            const long long off = ((long long)n * P + pos) * Cd + c0 + cc * 4;
             *reinterpret_cast<float4 *>(xh + off) = make_float4(0.f, 0.f, 0.f, 0.f);
             *reinterpret_cast<float4 *>(xl + off) = make_float4(0.f, 0.f, 0.f, 0.f);
         }
@@ -381,7 +383,7 @@ __global__ void __launch_bounds__(256) nchw_to_padded_f32_kernel(const float *__
         const int q = task & 7, sp = task >> 3;
         const long long s = s0 + sp;
         const int c = c0 + 4 * q;
-        if (s >= S || c >= C) continue;
+        if (s >= S || c >= Cd) continue;   // channels C..Cd of the row are zeros
         const int iz = (int)s / (int)HW;   // S < 2^31
         const int rem = (int)s - iz * (int)HW;
         const int iy = rem / W, ix = rem - iy * W;
@@ -389,7 +391,7 @@ __global__ void __launch_bounds__(256) nchw_to_padded_f32_kernel(const float *__
         if (zp < 0 || zp >= g.HZ || yp < 0 || yp >= HY || xq < 0 || xq >= HX) continue;
         const float4 v = make_float4(tile[4 * q][sp], tile[4 * q + 1][sp], tile[4 * q + 2][sp], tile[4 * q + 3][sp]);
         const float4 hi = make_float4(tf32_high(v.x), tf32_high(v.y), tf32_high(v.z), tf32_high(v.w));
-        const long long off = ((long long)n * P + zp * P2 + (long long)yp * HX + xq) * C + c;
+        const long long off = ((long long)n * P + zp * P2 + (long long)yp * HX + xq) * Cd + c;
         *reinterpret_cast<float4 *>(xh + off) = hi;
         *reinterpret_cast<float4 *>(xl + off) = make_float4(v.x - hi.x, v.y - hi.y, v.z - hi.z, v.w - hi.w);
     }
@@ -895,7 +897,11 @@ int round_up(int v, int m) { return (v + m - 1) / m * m; }
 bool build_pair_tables(const Plan &p, PairTables &T) {
     if ((p.dtype != CT_F16 && p.dtype != CT_F32) || p.G != 1 || !p.tabled) return false;
     // rows of the channels-last copy must be 16-byte multiples for TMA
-    if (p.C < 1 || p.C % (p.dtype == CT_F16 ? 8 : 4) != 0 || p.M < 1 || p.M > 16384 || p.N < 1 || p.N > 65535)
+    // channels-last rows must be 16-byte multiples for TMA: a channels-last X
+    // must already have them; the channels-first re-layout pads with zeros
+    const int row_elems = p.dtype == CT_F16 ? 8 : 4;
+    if (p.C < 1 || (p.layout == CT_NHWC && p.C % row_elems != 0) || p.M < 1 || p.M > 16384 || p.N < 1 ||
+        p.N > 65535)
         return false;
     for (int a = 0; a < 3; ++a)
         if (p.in[a] < 1 || p.in[a] > (1 << 24) || p.out[a] > (1 << 24)) return false;
@@ -910,6 +916,7 @@ bool build_pair_tables(const Plan &p, PairTables &T) {
     T.BL = (T.n_mt * T.Mt + 31) / 32 * 32;
     T.f32 = p.dtype == CT_F32;
     T.nhwc = p.layout == CT_NHWC;
+    T.Cd = (int32_t)ceil_div(p.C, row_elems) * row_elems;
     T.parts = T.f32 ? 2 : 1;
     T.cpb = T.f32 ? 32 : 64;
     T.KB = (int32_t)ceil_div(p.C, T.cpb);
@@ -999,6 +1006,7 @@ bool build_pair_tables(const Plan &p, PairTables &T) {
     const long long plane_pos = (long long)T.nJ[1] * HX;
     T.PU = (int32_t)ceil_div(plane_pos, 256);
     if ((long long)T.N * HZ * HY * HX + T.slice_rows + 256 >= (1LL << 31)) return false;
+    if ((long long)T.N * HZ * HY * HX * T.Cd >= (1LL << 40)) return false;
     const long long units = (long long)T.N * T.nJ[0] * T.PU * ng * T.n_mt;
     if (units > (1LL << 30)) return false;
     T.n_units = (int32_t)units;
@@ -1199,7 +1207,7 @@ size_t dense_pair_packed_bytes(const Plan &p) { return (size_t)ptables(p).n_mt *
 
 size_t dense_pair_ws_bytes(const Plan &p) {
     const PairTables &T = ptables(p);
-    return (size_t)T.parts * T.N * T.HZ * T.HY * T.HX * T.C * (T.f32 ? 4 : 2);
+    return (size_t)T.parts * T.N * T.HZ * T.HY * T.HX * T.Cd * (T.f32 ? 4 : 2);
 }
 
 ct_status dense_pair_prepack(const Plan &p, const void *w, void *wp, cudaStream_t st) {
@@ -1224,6 +1232,7 @@ ct_status dense_pair_run(const Plan &p, const void *x, const void *wp, const voi
         const long long tiles = ceil_div(S, kPadS);
         PadGeo g;
         g.C = T.C;
+        g.Cd = T.Cd;
         g.D = T.in[0];
         g.H = T.in[1];
         g.W = T.in[2];
@@ -1235,10 +1244,10 @@ ct_status dense_pair_run(const Plan &p, const void *x, const void *wp, const voi
         g.ox = -T.emin[2];
         // about 8 halo stores per thread
         g.halo_blocks = (int)std::max<long long>(1, std::min<long long>(1024, ceil_div(halo_count(g).n_all * 8, 2048)));
-        if (tiles + g.halo_blocks > 0x7fffffffLL || ceil_div(T.C, T.cpb) > 65535 || S >= (1LL << 31))
+        if (tiles + g.halo_blocks > 0x7fffffffLL || ceil_div(T.Cd, T.cpb) > 65535 || S >= (1LL << 31))
             return CT_ERR_UNSUPPORTED;
-        dim3 grid((unsigned)(tiles + g.halo_blocks), (unsigned)ceil_div(T.C, T.cpb), (unsigned)T.N);
-        const size_t plane_elems = (size_t)T.N * T.HZ * T.HY * T.HX * T.C;
+        dim3 grid((unsigned)(tiles + g.halo_blocks), (unsigned)ceil_div(T.Cd, T.cpb), (unsigned)T.N);
+        const size_t plane_elems = (size_t)T.N * T.HZ * T.HY * T.HX * T.Cd;
         if (T.nhwc) {
             // channels-last X: a padding copy of 16-byte pieces, about 8 per thread
             const long long pieces = (long long)T.C / (T.f32 ? 4 : 8);
@@ -1266,8 +1275,8 @@ ct_status dense_pair_run(const Plan &p, const void *x, const void *wp, const voi
         // remainders as two planes of the workspace
         const size_t eb = T.f32 ? 4 : 2;
         const cuuint64_t rows = (cuuint64_t)T.N * T.HZ * T.HY * T.HX;
-        const cuuint64_t dims[3] = {(cuuint64_t)T.C, rows, (cuuint64_t)T.parts};
-        const cuuint64_t strides[2] = {(cuuint64_t)T.C * eb, (cuuint64_t)(rows * T.C * eb)};
+        const cuuint64_t dims[3] = {(cuuint64_t)T.Cd, rows, (cuuint64_t)T.parts};
+        const cuuint64_t strides[2] = {(cuuint64_t)T.Cd * eb, (cuuint64_t)(rows * T.Cd * eb)};
         const cuuint32_t box[3] = {(cuuint32_t)T.cpb, (cuuint32_t)T.chunk_rows, 1};
         const cuuint32_t es[3] = {1, 1, 1};
         if (enc(&tmA, T.f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, ws, dims, strides,
