@@ -189,3 +189,59 @@ def test_run_argument_checks_without_device():
         assert e.value.status == 5
     finally:
         ct.ct_plan_destroy(plan)
+
+
+def _kernel_for(x_shape, w_shape, dtype, layout="nchw", strides=None, pads=None, group=1):
+    case = dict(x_shape=x_shape, w_shape=w_shape, strides=strides or [2] * (len(x_shape) - 2),
+                pads=pads, group=group, bias=True)
+    plan = ct.ct_plan(_desc_from_case(case, layout=layout, dtype=dtype))
+    try:
+        return (ct.ct_plan_kernel(plan), ct.ct_workspace_bytes(plan),
+                ct.ct_prepacked_weight_bytes(plan))
+    finally:
+        ct.ct_plan_destroy(plan)
+
+
+@pytest.mark.parametrize("x_shape,w_shape,dtype,layout,kernel", [
+    # tiny problems: one gather launch
+    ([1, 8, 8, 8], [8, 4, 3, 3], torch.float32, "nchw", "generic"),
+    # fp16 dense, channels-first, one or two axes: the CTA-pair kernel
+    ([8, 256, 64, 64], [256, 128, 4, 4], torch.float16, "nchw", "dense_tc_pair"),
+    ([4, 64, 3000], [64, 32, 16], torch.float16, "nchw", "dense_tc_pair"),
+    # fp16 dense, 3-D or channels-last: the single-SM halo kernel
+    ([2, 64, 32, 32, 32], [64, 32, 3, 3, 3], torch.float16, "nchw", "dense_tc"),
+    ([8, 256, 64, 64], [256, 128, 4, 4], torch.float16, "nhwc", "dense_tc"),
+    # more than 256 output channels, or channels that do not fill a 16-byte
+    # row: only the pair kernel takes them
+    ([2, 64, 8, 8, 8], [64, 320, 3, 3, 3], torch.float16, "nchw", "dense_tc_pair"),
+    ([8, 256, 32, 32], [256, 512, 4, 4], torch.float16, "nchw", "dense_tc_pair"),
+    ([4, 3, 40, 48], [3, 64, 4, 4], torch.float16, "nchw", "dense_tc_pair"),
+    # fp32: 3xTF32 on the pair kernel, both layouts
+    ([16, 512, 2048], [512, 256, 16], torch.float32, "nchw", "dense_tc_pair"),
+    ([16, 512, 2048], [512, 256, 16], torch.float32, "nhwc", "dense_tc_pair"),
+])
+def test_kernel_selection(x_shape, w_shape, dtype, layout, kernel):
+    """Automatic kernel choice for the shape classes each kernel was measured
+    fastest on (pure host code: no device touched)."""
+    got, ws, wb = _kernel_for(x_shape, w_shape, dtype, layout)
+    assert got == kernel, (x_shape, w_shape, dtype, layout, got)
+    assert wb > 0 and ws >= 0
+
+
+def test_pair_kernel_sizes():
+    """Workspace and packed-weight sizes of the pair kernel: the padded
+    channels-last copy (two planes for fp32) and one packed tile per
+    256 output channels."""
+    # 2-D decoder: 8 images x (64+2) x (64+2) padded positions x 256 channels x 2 bytes
+    kern, ws, wb = _kernel_for([8, 256, 64, 64], [256, 128, 4, 4], torch.float16)
+    assert kern == "dense_tc_pair" and ws == 8 * 66 * 66 * 256 * 2
+    # the same with 512 output channels: two channel tiles of packed weights
+    kern2, ws2, wb2 = _kernel_for([8, 256, 64, 64], [256, 256, 4, 4], torch.float16)
+    kern3, ws3, wb3 = _kernel_for([8, 256, 64, 64], [256, 512, 4, 4], torch.float16)
+    assert kern3 == "dense_tc_pair" and ws3 == ws2 and wb3 == 2 * wb2
+    # fp32: high parts and remainders of X (2 planes of 4-byte elements) and of W
+    kf, wsf, wbf = _kernel_for([8, 256, 64, 64], [256, 128, 4, 4], torch.float32)
+    assert kf == "dense_tc_pair" and wsf == 2 * 2 * ws and wbf == 2 * 2 * wb
+    # C = 3 is padded to an 8-channel (16-byte) row in the workspace
+    kc, wsc, _ = _kernel_for([4, 3, 40, 48], [3, 64, 4, 4], torch.float16)
+    assert kc == "dense_tc_pair" and wsc == 4 * 42 * 50 * 8 * 2
