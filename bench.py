@@ -286,29 +286,57 @@ class _Null:
 
 def time_e2e(wl, device, steps, warmup):
     """Through the public API with host buffers: pinned X -> device, ct_run,
-    Y -> pinned host, all inside the timed region every step."""
+    Y -> pinned host, all inside the timed region every step.  Steps are
+    pipelined the way a caller streaming batches would run them: copy-in,
+    compute and copy-out each on their own stream with two buffer sets, so
+    step i's input copy overlaps step i-1's compute and step i-2's output
+    copy (PCIe carries both directions at once)."""
     op, x_cpu = build_op(wl, device)
     xh = x_cpu.pin_memory()
-    yh = torch.empty(op.y_shape, dtype=wl.dtype).pin_memory()
-    xd = torch.empty_like(x_cpu, device=device)
-    yd = torch.empty(op.y_shape, dtype=wl.dtype, device=device)
+    yh = [torch.empty(op.y_shape, dtype=wl.dtype).pin_memory() for _ in range(2)]
+    xd = [torch.empty_like(x_cpu, device=device) for _ in range(2)]
+    yd = [torch.empty(op.y_shape, dtype=wl.dtype, device=device) for _ in range(2)]
+    s_in, s_run, s_out = (torch.cuda.Stream(device) for _ in range(3))
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_run = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    used = [False, False]
 
-    def step():
-        xd.copy_(xh, non_blocking=True)
-        op(xd, out=yd)
-        yh.copy_(yd, non_blocking=True)
+    def step(i):
+        b = i & 1
+        with torch.cuda.stream(s_in):
+            if used[b]:
+                s_in.wait_event(ev_run[b])   # the compute that read xd[b] is done
+            xd[b].copy_(xh, non_blocking=True)
+            ev_in[b].record(s_in)
+        with torch.cuda.stream(s_run):
+            s_run.wait_event(ev_in[b])
+            if used[b]:
+                s_run.wait_event(ev_out[b])  # yd[b] has been copied out
+            op(xd[b], out=yd[b], stream=s_run)
+            ev_run[b].record(s_run)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_run[b])
+            yh[b].copy_(yd[b], non_blocking=True)
+            ev_out[b].record(s_out)
+        used[b] = True
 
-    for _ in range(warmup):
-        step()
+    main = torch.cuda.current_stream(device)
+    for i in range(warmup):
+        step(i)
     torch.cuda.synchronize(device)
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
-    start.record()
-    for _ in range(steps):
-        step()
-    end.record()
+    start.record(main)
+    for st in (s_in, s_run, s_out):
+        st.wait_event(start)
+    for i in range(steps):
+        step(warmup + i)
+    for st in (s_in, s_run, s_out):
+        main.wait_stream(st)
+    end.record(main)
     torch.cuda.synchronize(device)
-    return start.elapsed_time(end), xh.numel() * xh.element_size(), yh.numel() * yh.element_size()
+    return start.elapsed_time(end), xh.numel() * xh.element_size(), yh[0].numel() * yh[0].element_size()
 
 
 # ---------------------------------------------------------------------------
