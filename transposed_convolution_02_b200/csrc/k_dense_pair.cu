@@ -1,17 +1,19 @@
-// Dense fp16 ConvTranspose (group 1, channels-first) on pairs of SMs: every
-// tcgen05 MMA spans the two CTAs of a cluster (cta_group::2, M = 256
-// positions).  Each SM reads its own 128 positions of A and only HALF of
-// every weight tile from its shared memory, and keeps the accumulators of its
-// 128 positions in its TMEM, double-buffered, so a unit's epilogue runs under
-// the next unit's MMAs.
+// Dense ConvTranspose (group 1, any rank, channels-first or channels-last;
+// fp16, or fp32 as 3xTF32) on pairs of SMs: every tcgen05 MMA spans the two
+// CTAs of a cluster (cta_group::2, M = 256 positions).  Each SM reads its own
+// 128 positions of A and only HALF of every weight tile from its shared
+// memory, and keeps the accumulators of its 128 positions in its TMEM,
+// double-buffered, so a unit's epilogue runs under the next unit's MMAs.
+// Output channels come in tiles of at most 256 (one MMA's N).
 //
 // Phases as in the halo kernel: output o = s*J + r per axis; tap k of phase r
 // reads input i = J + e, e = (r + pad_begin - k*d) / s (ai.onnx.ConvTranspose
 // README, implementation notes on the tap-reversed stride-1 form and the
 // grouped stride-phase variant).
 //
-// Input staging: X is re-laid into a zero-padded channels-last copy
-// Xp[n][zp][yp][xp][c], zp = iz - emin_z, yp = iy - emin_y, xp = ix - emin_x
+// Input staging: X is re-laid (channels-first) or copied (channels-last)
+// into a zero-padded channels-last copy Xp[n][zp][yp][xp][c] with c padded to
+// a 16-byte row, zp = iz - emin_z, yp = iy - emin_y, xp = ix - emin_x
 // (emin the smallest input offset of any tap per axis), HX = nJx + span_x
 // columns, HY = nJy + span_y rows and HZ = nJz + span_z slices per image.
 // Output position (Jy, Jx) of slice Jz is numbered F = Jy*HX + Jx, and its
