@@ -389,6 +389,81 @@ def oracle_sample(wl, target_s=12.0):
 
 # ---------------------------------------------------------------------------
 
+# Shapes beyond the five workloads: the stride-1 implicit GEMM (a 3x3
+# convolution with tap-reversed weights), the 1x1 stride-1 GEMM, channels-last
+# input, more than 256 output channels, 3 input channels, fp32 in 2-D.
+GENERAL_SHAPES = [
+    ("stride-1 3x3 fp16 X[8,256,64,64] W[256,256,3,3] p1", [8, 256, 64, 64], [256, 256, 3, 3],
+     torch.float16, "nchw", dict(strides=[1, 1], pads=[1, 1, 1, 1])),
+    ("1x1 stride-1 fp16 X[8,512,64,64] W[512,256,1,1]", [8, 512, 64, 64], [512, 256, 1, 1],
+     torch.float16, "nchw", dict(strides=[1, 1])),
+    ("channels-last decoder fp16 X[8,64,64,256] W[256,4,4,128] s2 p1", [8, 256, 64, 64], [256, 128, 4, 4],
+     torch.float16, "nhwc", dict(strides=[2, 2], pads=[1, 1, 1, 1])),
+    ("512-channel decoder fp16 X[8,256,32,32] W[256,512,4,4] s2 p1", [8, 256, 32, 32], [256, 512, 4, 4],
+     torch.float16, "nchw", dict(strides=[2, 2], pads=[1, 1, 1, 1])),
+    ("3-channel input fp16 X[16,3,128,128] W[3,64,4,4] s2 p1", [16, 3, 128, 128], [3, 64, 4, 4],
+     torch.float16, "nchw", dict(strides=[2, 2], pads=[1, 1, 1, 1])),
+    ("2-D fp32 decoder X[8,256,64,64] W[256,128,4,4] s2 p1", [8, 256, 64, 64], [256, 128, 4, 4],
+     torch.float32, "nchw", dict(strides=[2, 2], pads=[1, 1, 1, 1])),
+]
+
+
+def general_shapes(device, peaks, runs=50, algos=("auto", "dense_tc", "dense_tc_pertap",
+                                                  "dense_tc_pair", "generic"), only=None):
+    """Device time per call of each general shape under each algorithm that
+    accepts it (CUDA events around a batch of calls, inputs rotated so the
+    outputs exceed L2): kernel, effective TFLOP/s and the roofline of the
+    binding resource (tensor peak for the dtype, 3xTF32 for fp32, or HBM for
+    the algorithmic bytes X + W + bias + Y)."""
+    torch.cuda.set_device(device)
+    for si, (name, xs, ws, dt, layout, kw) in enumerate(GENERAL_SHAPES):
+        if only is not None and si != only:
+            continue
+        g = torch.Generator(device="cpu").manual_seed(7)
+        x = torch.randn(xs, generator=g).to(dt)
+        w = (torch.randn(ws, generator=g) / math.sqrt(ws[0] * math.prod(ws[2:]))).to(dt)
+        b = (torch.randn(ws[1], generator=g) * 0.1).to(dt)
+        if layout == "nhwc":
+            x = x.movedim(1, -1).contiguous()
+            w = w.movedim(1, -1).contiguous()
+        flop = 2 * xs[0] * xs[1] * ws[1] * math.prod(xs[2:]) * math.prod(ws[2:])
+        for algo in algos:
+            try:
+                op = ct.ConvTranspose(w.to(device), list(x.shape), b.to(device), layout=layout,
+                                      algo=algo, **kw)
+            except ct.CtError:
+                continue
+            if algo != "auto" and op.kernel != algo:
+                continue
+            esz = x.element_size()
+            ybytes = math.prod(op.y_shape) * esz
+            nbytes = (x.numel() + w.numel() + b.numel()) * esz + ybytes
+            sets = max(2, min(8, int(2 * 126 * 2 ** 20 // max(1, ybytes)) + 1))
+            xd = [x.to(device) for _ in range(sets)]
+            yd = [torch.empty(op.y_shape, dtype=dt, device=device) for _ in range(sets)]
+            for i in range(5):
+                op(xd[i % sets], out=yd[i % sets])
+            torch.cuda.synchronize(device)
+            s0 = torch.cuda.Event(enable_timing=True)
+            s1 = torch.cuda.Event(enable_timing=True)
+            s0.record()
+            for i in range(runs):
+                op(xd[i % sets], out=yd[i % sets])
+            s1.record()
+            torch.cuda.synchronize(device)
+            us = s0.elapsed_time(s1) * 1e3 / runs
+            tc_peak = peaks["tc_tflops"] * (TF32_PER_BF16 / 3 if dt == torch.float32 else 1.0)
+            t_tc = flop / (tc_peak * 1e12)
+            t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+            bound = "tensor" if t_tc >= t_hbm else "hbm"
+            frac = max(t_tc, t_hbm) / (us * 1e-6)
+            print(json.dumps({"shape": name, "algo": algo, "kernel": op.kernel,
+                              "us_per_call": round(us, 2), "tflops": round(flop / us / 1e6, 1),
+                              "gbs": round(nbytes / us / 1e3, 1), "bound": bound,
+                              "frac": round(frac, 3)}), flush=True)
+            del op, xd, yd
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -401,6 +476,13 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--plain", action="store_true",
                     help="profiling mode: eager ct_run launches of one workload, nothing else")
+    ap.add_argument("--general", action="store_true",
+                    help="time a set of general shapes (stride 1, 1x1, channels-last, many or few "
+                         "channels) and print one JSON line per shape")
+    ap.add_argument("--shape", type=int, default=None,
+                    help="with --general: time only this entry of the general shape list")
+    ap.add_argument("--algo", default=None, help="with --general: time only this algorithm")
+    ap.add_argument("--runs", type=int, default=50, help="with --general: timed calls per shape")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -438,6 +520,13 @@ def main():
                 "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
+        return
+
+    if args.general:
+        kw = dict(runs=args.runs, only=args.shape)
+        if args.algo:
+            kw["algos"] = (args.algo,)
+        general_shapes(torch.device("cuda", local), load_peaks(), **kw)
         return
 
     if args.plain:
