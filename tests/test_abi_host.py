@@ -245,3 +245,29 @@ def test_pair_kernel_sizes():
     # C = 3 is padded to an 8-channel (16-byte) row in the workspace
     kc, wsc, _ = _kernel_for([4, 3, 40, 48], [3, 64, 4, 4], torch.float16)
     assert kc == "dense_tc_pair" and wsc == 4 * 42 * 50 * 8 * 2
+
+
+def test_general_shapes_plan_to_tensor_core_kernels():
+    """Every shape ``bench.py --general`` times plans (host code only) to a
+    tensor-core kernel: stride 1 with a 3x3 window and 1x1 (the tap-reversed
+    stride-1 form and the plain GEMM), channels-last, more than 256 output
+    channels, a 3-channel input and fp32."""
+    import bench
+
+    assert len(bench.GENERAL_SHAPES) >= 6
+    for name, xs, ws, dt, layout, kw in bench.GENERAL_SHAPES:
+        xsl = xs if layout == "nchw" else [xs[0]] + xs[2:] + [xs[1]]
+        wsl = ws if layout == "nchw" else [ws[0]] + ws[2:] + [ws[1]]
+        desc = ct.make_desc(xsl, wsl, dtype=dt, layout=layout, bias_len=ws[1], **kw)
+        plan = ct.ct_plan(desc)
+        try:
+            kern = ct.ct_plan_kernel(plan)
+            y_shape, _, _ = ct.ct_output_shape(desc)
+        finally:
+            ct.ct_plan_destroy(plan)
+        assert kern in ("dense_tc_pair", "dense_tc"), (name, kern)
+        # spatial sizes: stride 1 keeps them (3x3 with pad 1, 1x1), stride 2
+        # with k = 4, p = 1 doubles them
+        sp = y_shape[2:] if layout == "nchw" else y_shape[1:-1]
+        mult = kw["strides"][0]
+        assert list(sp) == [mult * v for v in xs[2:]], (name, y_shape)

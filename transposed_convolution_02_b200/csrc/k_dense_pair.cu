@@ -898,9 +898,9 @@ int round_up(int v, int m) { return (v + m - 1) / m * m; }
 
 bool build_pair_tables(const Plan &p, PairTables &T) {
     if ((p.dtype != CT_F16 && p.dtype != CT_F32) || p.G != 1 || !p.tabled) return false;
-    // rows of the channels-last copy must be 16-byte multiples for TMA
-    // channels-last rows must be 16-byte multiples for TMA: a channels-last X
-    // must already have them; the channels-first re-layout pads with zeros
+    // rows of the channels-last copy must be 16-byte multiples for TMA: a
+    // channels-last X must already have them; the channels-first re-layout
+    // pads with zeros
     const int row_elems = p.dtype == CT_F16 ? 8 : 4;
     if (p.C < 1 || (p.layout == CT_NHWC && p.C % row_elems != 0) || p.M < 1 || p.M > 16384 || p.N < 1 ||
         p.N > 65535)
