@@ -464,3 +464,20 @@ def test_dense_tc_pair_channels_padded(dtype, case):
     channels-first re-layout pads them with zeros; automatic selection takes
     the pair kernel instead of the generic one."""
     full_parity(case, dtype, 87, "nchw", expect_kernel="dense_tc_pair")
+
+
+@pytest.mark.parametrize("idx", range(6))
+def test_general_shapes_sampled(idx):
+    """The shapes ``bench.py --general`` times (stride-1 3x3, 1x1, channels-last,
+    512 output channels, 3 input channels, fp32 2-D), at the timed size and
+    with the automatically chosen kernel: sampled outputs against the oracle."""
+    import bench
+
+    name, xs, ws, dt, layout, kw = bench.GENERAL_SHAPES[idx]
+    case = dict(x_shape=list(xs), w_shape=list(ws), strides=kw["strides"], pads=kw.get("pads"),
+                bias=True)
+    x, w, b = draw_case(case, dt, 900 + 10 * idx, layout)
+    op, y = gpu_run(case, x, w, b, layout, "auto")
+    assert op.kernel in ("dense_tc_pair", "dense_tc"), (name, op.kernel)
+    assert not torch.isnan(y).any(), name
+    sampled_parity(op, y, x, w, b, case, dt, layout, np.random.default_rng(idx), n_random=600)
