@@ -138,7 +138,11 @@ typedef struct ct_plan_s ct_plan_t;
 /* Resolve the output: Y's dims in the descriptor's layout (rank + 2 entries)
  * and the begin/end pads per axis.  Pure host code, no device touched.
  * Implements the output-size rule above with the auto_pad / output_shape /
- * output_padding rows of the README's "Attributes" table. */
+ * output_padding rows of the README's "Attributes" table.  Library limits
+ * (CT_ERR_ATTR beyond them, so that no size arithmetic overflows int64):
+ * N, C, M/group, group, every spatial size, kernel size, stride, dilation,
+ * pad and requested output size at most 2^30 in magnitude; X, W and Y each
+ * at most 2^60 elements. */
 CT_API ct_status ct_output_shape(const ct_desc *desc, int64_t y_dims[5],
                           int64_t pad_begin[3], int64_t pad_end[3]);
 

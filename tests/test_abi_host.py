@@ -271,3 +271,31 @@ def test_general_shapes_plan_to_tensor_core_kernels():
         sp = y_shape[2:] if layout == "nchw" else y_shape[1:-1]
         mult = kw["strides"][0]
         assert list(sp) == [mult * v for v in xs[2:]], (name, y_shape)
+
+
+def test_size_limits_reject_overflowing_descriptors():
+    """Sizes whose arithmetic would overflow int64 are refused at resolve
+    time (CT_ERR_ATTR = 4); sizes just inside the limits resolve."""
+    big = 1 << 30
+
+    def status(x_shape, w_shape, **kw):
+        d = ct.make_desc(x_shape, w_shape, dtype=torch.float16, **kw)
+        try:
+            ct.ct_output_shape(d)
+            return 0
+        except ct.CtError as e:
+            return e.status
+
+    assert status([1, 1, big], [1, 1, 1], strides=[1]) == 0
+    assert status([1, 1, big + 1], [1, 1, 1], strides=[1]) == 4
+    assert status([1, 1, 4], [1, 1, 1], strides=[big + 1]) == 4
+    assert status([1, 1, 4], [1, 1, 3], strides=[1], dilations=[1 << 40]) == 4
+    assert status([1, 1, 4], [1, 1, 3], strides=[1], pads=[-(1 << 40), 0]) == 4
+    assert status([1 << 31, 1, 4], [1, 1, 3], strides=[1]) == 4
+    assert status([1, 1, 4], [1, 1 << 31, 3], strides=[1]) == 4
+    # each size in range, but X has 2^30 * 2^30 * 2^30 elements
+    assert status([big, big, big], [big, 1, 1], strides=[1]) == 4
+    # Y too large: 2^20 images x 2^20 channels x 2^30 outputs
+    assert status([1 << 20, 1, 1 << 29], [1, 1 << 20, 1], strides=[2], output_padding=[1]) == 4
+    # the old overflow: s * (in - 1) near 2^62 now refused instead of wrapping
+    assert status([1, 1, 1 << 31], [1, 1, 1], strides=[1 << 31]) == 4

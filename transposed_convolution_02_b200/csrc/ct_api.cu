@@ -31,6 +31,19 @@ void split_total(int64_t total, bool odd_at_end, int64_t *pb, int64_t *pe) {
     }
 }
 
+// Size limits that keep every product below in int64: a batch, channel,
+// group, spatial size, kernel size, stride, dilation, pad or requested output
+// size at most 2^30 in magnitude, and at most 2^60 elements in X, W or Y.
+constexpr int64_t kMaxDim = int64_t(1) << 30;
+constexpr int64_t kMaxElems = int64_t(1) << 60;
+
+// a * b when both are in [0, kMaxElems] and so is the product, else -1
+int64_t mul_capped(int64_t a, int64_t b) {
+    if (a < 0 || b < 0) return -1;
+    if (a != 0 && b > kMaxElems / a) return -1;
+    return a * b;
+}
+
 // Validate and resolve a descriptor into a plan's geometry.
 ct_status resolve(const ct_desc *d, Plan *p) {
     if (!d) return CT_ERR_NULL;
@@ -41,11 +54,12 @@ ct_status resolve(const ct_desc *d, Plan *p) {
     if (d->algo < CT_ALGO_AUTO || d->algo > CT_ALGO_DENSE_TC_PAIR) return CT_ERR_ATTR;
     if (d->activation != CT_ACT_IDENTITY && d->activation != CT_ACT_RELU) return CT_ERR_ATTR;
     const int r = d->rank;
-    if (d->N < 0 || d->C < 0) return CT_ERR_ATTR;
+    if (d->N < 0 || d->C < 0 || d->N > kMaxDim || d->C > kMaxDim) return CT_ERR_ATTR;
     if (d->group <= 0 || d->C % d->group != 0) return CT_ERR_CHANNELS;
     if (d->w_dims[0] != d->C) return CT_ERR_CHANNELS;
     const int64_t mg = d->layout == CT_NCHW ? d->w_dims[1] : d->w_dims[r + 1];
     if (mg <= 0) return CT_ERR_CHANNELS;
+    if (mg > kMaxDim || d->group > kMaxDim) return CT_ERR_ATTR;
     const int64_t M = mg * d->group;
     if (d->bias_len < 0 || (d->bias_len != 0 && d->bias_len != M)) return CT_ERR_CHANNELS;
 
@@ -70,6 +84,12 @@ ct_status resolve(const ct_desc *d, Plan *p) {
         dl[a] = d->dilations[a];
         op[a] = d->output_padding[a];
         if (s[a] <= 0 || dl[a] <= 0 || k[a] <= 0 || in[a] < 0) return CT_ERR_ATTR;
+        if (s[a] > kMaxDim || dl[a] > kMaxDim || k[a] > kMaxDim || in[a] > kMaxDim) return CT_ERR_ATTR;
+        if (d->pads[a] < -kMaxDim || d->pads[a] > kMaxDim || d->pads[r + a] < -kMaxDim ||
+            d->pads[r + a] > kMaxDim)
+            return CT_ERR_ATTR;
+        if (d->has_output_shape && (d->output_shape[a] < -kMaxDim || d->output_shape[a] > kMaxDim))
+            return CT_ERR_ATTR;
         const int64_t lim = s[a] > dl[a] ? s[a] : dl[a];
         if (op[a] < 0 || op[a] >= lim) return CT_ERR_ATTR;
         if (d->has_kernel_shape && d->kernel_shape[a] != k[a]) return CT_ERR_ATTR;
@@ -101,6 +121,14 @@ ct_status resolve(const ct_desc *d, Plan *p) {
         out[a] = natural[a] - pb[a] - pe[a];
         if (out[a] <= 0) return CT_ERR_ATTR;
     }
+    // element counts of X, W and Y
+    int64_t nx = mul_capped(d->N, d->C), nw = mul_capped(d->C, mg), ny = mul_capped(d->N, M);
+    for (int a = 0; a < r; ++a) {
+        nx = mul_capped(nx, in[a]);
+        nw = mul_capped(nw, k[a]);
+        ny = mul_capped(ny, out[a]);
+    }
+    if (nx < 0 || nw < 0 || ny < 0) return CT_ERR_ATTR;
     // pad to three axes, the given ones innermost
     for (int a = 0; a < 3; ++a) {
         const int src = a - (3 - r);
