@@ -299,3 +299,11 @@ def test_size_limits_reject_overflowing_descriptors():
     assert status([1 << 20, 1, 1 << 29], [1, 1 << 20, 1], strides=[2], output_padding=[1]) == 4
     # the old overflow: s * (in - 1) near 2^62 now refused instead of wrapping
     assert status([1, 1, 1 << 31], [1, 1, 1], strides=[1 << 31]) == 4
+
+
+def test_ignored_pads_are_not_range_checked():
+    """With output_shape the explicit pads are ignored, whatever their size."""
+    d = ct.make_desc([1, 1, 4], [1, 1, 3], dtype=torch.float16, strides=[2],
+                     pads=[1 << 40, 0], output_shape=[9])
+    y, pb, pe = ct.ct_output_shape(d)
+    assert list(y) == [1, 1, 9] and (pb[0], pe[0]) == (0, 0)

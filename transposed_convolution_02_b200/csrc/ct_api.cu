@@ -85,8 +85,9 @@ ct_status resolve(const ct_desc *d, Plan *p) {
         op[a] = d->output_padding[a];
         if (s[a] <= 0 || dl[a] <= 0 || k[a] <= 0 || in[a] < 0) return CT_ERR_ATTR;
         if (s[a] > kMaxDim || dl[a] > kMaxDim || k[a] > kMaxDim || in[a] > kMaxDim) return CT_ERR_ATTR;
-        if (d->pads[a] < -kMaxDim || d->pads[a] > kMaxDim || d->pads[r + a] < -kMaxDim ||
-            d->pads[r + a] > kMaxDim)
+        if (!d->has_output_shape &&   // with output_shape the pads are ignored
+            (d->pads[a] < -kMaxDim || d->pads[a] > kMaxDim || d->pads[r + a] < -kMaxDim ||
+             d->pads[r + a] > kMaxDim))
             return CT_ERR_ATTR;
         if (d->has_output_shape && (d->output_shape[a] < -kMaxDim || d->output_shape[a] > kMaxDim))
             return CT_ERR_ATTR;
