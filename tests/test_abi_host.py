@@ -307,3 +307,28 @@ def test_ignored_pads_are_not_range_checked():
                      pads=[1 << 40, 0], output_shape=[9])
     y, pb, pe = ct.ct_output_shape(d)
     assert list(y) == [1, 1, 9] and (pb[0], pe[0]) == (0, 0)
+
+
+def test_call_checks_refuse_mismatched_tensors():
+    """The binding refuses X or Y that do not match the plan before any launch
+    (host logic only; CPU tensors stand in for device ones)."""
+    dev = torch.device("cpu")
+    x = torch.zeros(2, 4, 5, dtype=torch.float16)
+    y = torch.zeros(2, 6, 9, dtype=torch.float16)
+    ct.check_io(x, None, [2, 4, 5], [2, 6, 9], torch.float16, dev)
+    ct.check_io(x, y, [2, 4, 5], [2, 6, 9], torch.float16, dev)
+    with pytest.raises(ValueError):
+        ct.check_io(torch.zeros(2, 4, 6, dtype=torch.float16), None, [2, 4, 5], [2, 6, 9],
+                    torch.float16, dev)
+    with pytest.raises(ValueError):
+        ct.check_io(x.float(), None, [2, 4, 5], [2, 6, 9], torch.float16, dev)
+    with pytest.raises(ValueError):
+        ct.check_io(x, torch.zeros(2, 6, 8, dtype=torch.float16), [2, 4, 5], [2, 6, 9],
+                    torch.float16, dev)
+    with pytest.raises(ValueError):
+        ct.check_io(x, y.float(), [2, 4, 5], [2, 6, 9], torch.float16, dev)
+    with pytest.raises(ValueError):
+        ct.check_io(x, torch.zeros(2, 9, 6, dtype=torch.float16).transpose(1, 2), [2, 4, 5],
+                    [2, 6, 9], torch.float16, dev)
+    with pytest.raises(ValueError):
+        ct.check_io(x, None, [2, 4, 5], [2, 6, 9], torch.float16, torch.device("meta"))

@@ -229,6 +229,22 @@ def _stream_ptr(stream):
     return ctypes.c_void_p(s.cuda_stream)
 
 
+def check_io(x, out, x_shape, y_shape, dtype, device):
+    """Refuse a call whose tensors do not match the plan (the kernels trust the
+    planned sizes: a different X or Y would be read or written out of bounds)."""
+    if list(x.shape) != list(x_shape):
+        raise ValueError("X has shape %s, the plan was made for %s" % (list(x.shape), list(x_shape)))
+    if x.dtype != dtype:
+        raise ValueError("X is %s, the plan computes in %s" % (x.dtype, dtype))
+    if x.device != device:
+        raise ValueError("X is on %s, the packed weights on %s" % (x.device, device))
+    if out is not None:
+        if list(out.shape) != list(y_shape) or out.dtype != dtype or out.device != device:
+            raise ValueError("out must be a %s tensor of shape %s on %s" % (dtype, list(y_shape), device))
+        if not out.is_contiguous():
+            raise ValueError("out must be contiguous")
+
+
 class ConvTranspose:
     """A planned ConvTranspose with its weight pre-packed on the device.
 
@@ -242,8 +258,12 @@ class ConvTranspose:
                  stream=None):
         if not w.is_cuda:
             raise ValueError("W must be a CUDA tensor")
+        if bias is not None and (bias.dtype != w.dtype or bias.device != w.device):
+            raise ValueError("bias must be a tensor of W's dtype on W's device")
         self.layout = layout
         self.dtype = w.dtype
+        self.device = w.device
+        self.x_shape = list(x_shape)
         self.desc = make_desc(list(x_shape), list(w.shape), dtype=w.dtype, layout=layout,
                               strides=strides, dilations=dilations, pads=pads,
                               output_padding=output_padding, auto_pad=auto_pad, group=group,
@@ -264,8 +284,9 @@ class ConvTranspose:
         self._w_keep = w
 
     def __call__(self, x, out=None, stream=None):
-        if x.dtype != self.dtype or not x.is_cuda:
-            raise ValueError("X must be a CUDA tensor of the weight's dtype")
+        if not x.is_cuda:
+            raise ValueError("X must be a CUDA tensor")
+        check_io(x, out, self.x_shape, self.y_shape, self.dtype, self.device)
         x = x.contiguous()
         y = out if out is not None else torch.empty(self.y_shape, dtype=self.dtype,
                                                     device=x.device)
@@ -274,7 +295,8 @@ class ConvTranspose:
         return y
 
     def run_ptrs(self, x_ptr, y_ptr, stream_ptr):
-        """Launch on raw device pointers (benchmark loops)."""
+        """Launch on raw device pointers (benchmark loops); the caller
+        guarantees buffers of the planned shapes, dtype and device."""
         ct_run(self.plan, x_ptr, _ptr(self.w_packed), _ptr(self.bias), y_ptr,
                _ptr(self.workspace), stream_ptr)
 
