@@ -206,6 +206,19 @@ CT_API void ct_plan_destroy(ct_plan_t *plan);
 /* Static, human-readable text for a status code. */
 CT_API const char *ct_status_string(ct_status status);
 
+/* Failure report of the kernels' bounded waits.  Every wait of the
+ * tensor-core and grouped kernels on an mbarrier gives up after about one
+ * second of SM clock; the kernel then records a code in its module's device
+ * error word, skips the rest of its work (so Y is not valid) and returns, and
+ * the device stays usable.  This call waits for `stream` (work that ran
+ * earlier on other streams must be finished by the caller), then reads and
+ * clears the error words of the current device.  *code = 0 and CT_OK when no
+ * wait ran out since the last call; otherwise *code = 100 * module + wait
+ * site (module 1 dense_tc, 2 dense_tc_pair, 3 dense_tc_pertap, 4 grouped)
+ * and CT_ERR_DEVICE.  CT_ERR_DEVICE with *code = 0 means a CUDA call failed
+ * (or the current device is not an sm_100 part). */
+CT_API ct_status ct_take_device_error(void *stream, int32_t *code);
+
 #ifdef __cplusplus
 }
 #endif

@@ -332,3 +332,16 @@ def test_call_checks_refuse_mismatched_tensors():
                     [2, 6, 9], torch.float16, dev)
     with pytest.raises(ValueError):
         ct.check_io(x, None, [2, 4, 5], [2, 6, 9], torch.float16, torch.device("meta"))
+
+
+def test_take_device_error_without_device():
+    """ct_take_device_error needs the device: without one it reports
+    CT_ERR_DEVICE (7) with no wait code."""
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    with pytest.raises(ct.CtError) as e:
+        ct.ct_take_device_error()
+    assert e.value.status == 7
+    code = ctypes.c_int32(-5)
+    assert ct.lib().ct_take_device_error(None, ctypes.byref(code)) == 7 and code.value == 0
+    assert ct.lib().ct_take_device_error(None, None) == 6          # CT_ERR_NULL

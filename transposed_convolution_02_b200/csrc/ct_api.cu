@@ -382,6 +382,23 @@ ct_status ct_run(const ct_plan_t *plan, const void *x, const void *w_packed, con
     }
 }
 
+ct_status ct_take_device_error(void *stream, int32_t *code) {
+    if (!code) return CT_ERR_NULL;
+    *code = 0;
+    ct_status st = check_device();
+    if (st != CT_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // module numbers 1..4: dense_tc, dense_tc_pair, dense_tc_pertap, grouped
+    const int words[4] = {dense_tc_take_error(s), dense_pair_take_error(s), dense_pertap_take_error(s),
+                          grouped_take_error(s)};
+    bool cuda_failed = false;
+    for (int i = 0; i < 4; ++i) {
+        if (words[i] < 0) cuda_failed = true;
+        if (words[i] > 0 && *code == 0) *code = (i + 1) * 100 + words[i];
+    }
+    return (cuda_failed || *code != 0) ? CT_ERR_DEVICE : CT_OK;
+}
+
 void ct_plan_destroy(ct_plan_t *plan) { delete reinterpret_cast<Plan *>(plan); }
 
 const char *ct_status_string(ct_status status) {

@@ -56,6 +56,26 @@ inline int sm_count() {
     return n;
 }
 
+// Read a module's device error word (set by a bounded wait that ran out) and
+// clear it, in order on `st`, then wait for `st`.  Returns the code read (0:
+// none), or -1 when a CUDA call failed.
+template <typename T>
+inline int take_error_word(T &symbol, cudaStream_t st) {
+    int v = 0;
+    const int zero = 0;
+    if (cudaMemcpyFromSymbolAsync(&v, symbol, sizeof(int), 0, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess) {
+        cudaGetLastError();
+        return -1;
+    }
+    if (v != 0 && (cudaMemcpyToSymbolAsync(symbol, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+                   cudaStreamSynchronize(st) != cudaSuccess)) {
+        cudaGetLastError();
+        return -1;
+    }
+    return v;
+}
+
 // Raise a kernel's dynamic shared-memory limit once per device.
 template <typename K>
 inline bool allow_smem(K kernel, std::atomic<int> *flags, int bytes) {

@@ -102,6 +102,14 @@ ct_status grouped_prepack(const Plan &p, const void *w, void *wp, cudaStream_t s
 ct_status grouped_run(const Plan &p, const void *x, const void *wp, const void *bias, void *y,
                       cudaStream_t st);
 
+// Device error words of the tensor-core and grouped modules: the code of a
+// bounded wait that ran out since the last read (0: none; -1: CUDA failed),
+// read in order on the stream and cleared.
+int dense_tc_take_error(cudaStream_t st);
+int dense_pertap_take_error(cudaStream_t st);
+int dense_pair_take_error(cudaStream_t st);
+int grouped_take_error(cudaStream_t st);
+
 // Map the last CUDA error to a status (and clear it).
 inline ct_status launch_status() {
     cudaError_t e = cudaGetLastError();

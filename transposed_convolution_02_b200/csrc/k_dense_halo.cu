@@ -895,4 +895,6 @@ ct_status dense_tc_run(const Plan &p, const void *x, const void *wp, const void 
     return launch_status();
 }
 
+int dense_tc_take_error(cudaStream_t st) { return take_error_word(g_dense_halo_err, st); }
+
 }  // namespace ct

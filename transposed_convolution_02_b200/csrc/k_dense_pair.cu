@@ -1313,4 +1313,6 @@ ct_status dense_pair_run(const Plan &p, const void *x, const void *wp, const voi
     return launch_pair<CT_ACT_IDENTITY, __half>(T, tmA, tmB, tmBs, bias, y, st);
 }
 
+int dense_pair_take_error(cudaStream_t st) { return take_error_word(g_dense_pair_err, st); }
+
 }  // namespace ct

@@ -494,4 +494,6 @@ ct_status dense_pertap_run(const Plan &p, const void *x, const void *wp, const v
     return launch_status();
 }
 
+int dense_pertap_take_error(cudaStream_t st) { return take_error_word(g_dense_pertap_err, st); }
+
 }  // namespace ct

@@ -766,4 +766,6 @@ ct_status grouped_run(const Plan &p, const void *x, const void *wp, const void *
     return CT_ERR_UNSUPPORTED;
 }
 
+int grouped_take_error(cudaStream_t st) { return take_error_word(g_grouped_err, st); }
+
 }  // namespace ct

@@ -33,7 +33,7 @@ ALGO = {"auto": 0, "generic": 1, "dense_tc": 2, "fp32_gemm": 3, "grouped": 4,
 EXPORTED = ["ct_output_shape", "ct_plan", "ct_plan_kernel", "ct_plan_launches",
             "ct_prepacked_weight_bytes",
             "ct_workspace_bytes", "ct_prepack_weights", "ct_run", "ct_run_noalloc",
-            "ct_plan_destroy", "ct_status_string"]
+            "ct_plan_destroy", "ct_status_string", "ct_take_device_error"]
 
 
 class CtError(RuntimeError):
@@ -83,10 +83,12 @@ def lib():
         L.ct_run_noalloc.argtypes = [P, P, P, P, P, P]
         L.ct_plan_destroy.argtypes = [P]
         L.ct_plan_destroy.restype = None
+        L.ct_take_device_error.argtypes = [P, ctypes.POINTER(ctypes.c_int32)]
         L.ct_status_string.argtypes = [ctypes.c_int]
         L.ct_status_string.restype = ctypes.c_char_p
         for name in ("ct_output_shape", "ct_plan", "ct_plan_launches", "ct_prepacked_weight_bytes",
-                     "ct_workspace_bytes", "ct_prepack_weights", "ct_run", "ct_run_noalloc"):
+                     "ct_workspace_bytes", "ct_prepack_weights", "ct_run", "ct_run_noalloc",
+                     "ct_take_device_error"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -163,6 +165,18 @@ def ct_run_noalloc(plan, x_ptr, wp_ptr, bias_ptr, y_ptr, stream):
     st = lib().ct_run_noalloc(plan, x_ptr, wp_ptr, bias_ptr, y_ptr, stream)
     if st != CT_OK:
         raise CtError(st, "ct_run_noalloc")
+
+
+def ct_take_device_error(stream=None):
+    """Wait for the stream, then read and clear the kernels' device error
+    words: 0 when no bounded wait ran out since the last call, else the code
+    100 * module + wait site.  Raises CtError when a CUDA call failed."""
+    code = ctypes.c_int32()
+    st = lib().ct_take_device_error(_stream_ptr(stream) if torch.cuda.is_available() else None,
+                                    ctypes.byref(code))
+    if st != CT_OK and code.value == 0:
+        raise CtError(st, "ct_take_device_error")
+    return code.value
 
 
 def ct_plan_destroy(plan):
