@@ -39,9 +39,6 @@
 #include "ct_internal.h"
 #include "sm100.cuh"
 
-#ifndef V_OPMINB
-#define V_OPMINB 3
-#endif
 namespace ct {
 
 __device__ int g_grouped_err;
@@ -214,13 +211,17 @@ __device__ __forceinline__ void one_phase_rows(const GroupedArgs &A, const uint4
     }
 }
 
+// Resident CTAs per SM the one-phase path is compiled for: the register cap
+// its launch bounds give the compiler.
+constexpr int kGOnePhaseMinBlocks = 3;
+
 // NSTEP > 0: the one-phase path -- one output channel tile (MT == 1), a
 // single stride phase with taps, s_x == 2, NSTEP (tap pair, k-step) steps
 // whose weight fragments and slab offsets stay in registers, and outputs
 // stored straight from the accumulators as (bias, value) pairs.
 // ACT: the output activation (ct_activation), fixed at compile time.
 template <int MT, int NSTEP, int ACT>
-__global__ void __launch_bounds__(kGThreads, NSTEP > 0 ? V_OPMINB : (MT <= 2 ? 4 : 2))
+__global__ void __launch_bounds__(kGThreads, NSTEP > 0 ? kGOnePhaseMinBlocks : (MT <= 2 ? 4 : 2))
     grouped_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ GroupedArgs A,
                    const __half *__restrict__ x, const uint4 *__restrict__ wp,
                    const __half *__restrict__ bias, __half *__restrict__ y) {
