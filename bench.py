@@ -11,9 +11,9 @@ the L2 holds between reuses).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-Under torchrun each rank runs its own replica of the workload (weak scaling:
-the batch is independent per GPU, no collective on the data path); the
-reported time is the max over ranks.  ``--impl reference`` times the fp64
+Under torchrun each rank takes its own workload-sized slice of the global
+batch (weak scaling: images are independent, no collective on the data
+path); the reported time is the max over ranks.  ``--impl reference`` times the fp64
 CPU oracle on a bounded sample of the same workload instead.
 """
 
@@ -494,7 +494,8 @@ def main():
     flop, nbytes = workload_numbers(wl)
     config = {"workload": wl.name, "x": list(wl.x_shape), "w": list(wl.w_shape),
               "y": list(wl.y_shape), "global_batch": wl.x_shape[0] * max(world, 1),
-              "parallelism": "dp%d (independent replica per GPU)" % max(world, 1)}
+              "parallelism": "dp%d (batch sharded: each GPU one workload-sized slice, "
+                             "no data-path collective)" % max(world, 1)}
 
     if args.impl == "reference":
         if rank != 0:
