@@ -345,3 +345,17 @@ def test_take_device_error_without_device():
     code = ctypes.c_int32(-5)
     assert ct.lib().ct_take_device_error(None, ctypes.byref(code)) == 7 and code.value == 0
     assert ct.lib().ct_take_device_error(None, None) == 6          # CT_ERR_NULL
+
+
+def test_binding_argument_counts_match_header():
+    """Every function include/ct.h declares is bound with as many ctypes
+    arguments as the declaration has parameters (guards binding drift)."""
+    L = ct.lib()
+    src = open(os.path.join(ROOT, "include", "ct.h")).read()
+    decls = re.findall(r"CT_API\s+[\w\s\*]*?\b(ct_\w+)\s*\(([^)]*)\)", src)
+    assert decls
+    for name, params in decls:
+        params = " ".join(params.split())
+        n = 0 if params in ("", "void") else params.count(",") + 1
+        assert getattr(L, name).argtypes is not None, name
+        assert len(getattr(L, name).argtypes) == n, (name, n, getattr(L, name).argtypes)
