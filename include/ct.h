@@ -26,7 +26,11 @@
  * "Type constraints").  All tensors are dense, row-major, in device memory.
  *
  * Ownership: the caller owns every device buffer and the stream; the library
- * owns only the opaque plan.  No entry point allocates device memory.
+ * owns only the opaque plan.  No entry point calls a device allocator; the
+ * device memory libct.so holds by itself is its code and its file-scope
+ * device arrays (the ct_run_noalloc workspace among them), which CUDA loads
+ * onto a device with the library's kernels, at the latest on the first call
+ * that uses that device.
  * Errors: every entry point returns a ct_status; nothing is thrown across the
  * ABI, nothing is printed.  Validation happens in ct_plan, before any launch.
  * The status classes mirror the error classes of ClikaRT::ops::conv_transpose
@@ -180,6 +184,27 @@ CT_API ct_status ct_prepack_weights(const ct_plan_t *plan, const void *w, void *
 CT_API ct_status ct_run(const ct_plan_t *plan, const void *x, const void *w_packed,
                  const void *bias, void *y, void *workspace, void *stream);
 
+/* Parts of one ct_run, for measuring them apart (ct_run_parts).  A call
+ * consists of preparation launches (the re-layout of X into the workspace,
+ * and the bias fill of outputs no tap reaches) followed by one main kernel
+ * (the phase GEMM or gather).  Plans whose call is a single kernel have no
+ * preparation: CT_PART_PREPARE alone launches nothing for them. */
+#define CT_PART_PREPARE 1
+#define CT_PART_MAIN 2
+#define CT_PART_ALL 3
+
+/* ct_run restricted to the parts in `parts` (a mask of CT_PART_*; 0 does
+ * nothing, other bits are CT_ERR_ATTR).  ct_run(...) is ct_run_parts(...,
+ * CT_PART_ALL).  CT_PART_MAIN alone reads the workspace and Y as an earlier
+ * CT_PART_PREPARE call with the same x, workspace and y left them: a
+ * benchmark prepares once and then times the main kernel by itself.  With
+ * anything else in the workspace the main kernel still reads and writes
+ * only inside the planned buffers, but Y is not the operator's result.
+ * Arguments, alignment and errors as for ct_run. */
+CT_API ct_status ct_run_parts(const ct_plan_t *plan, const void *x, const void *w_packed,
+                              const void *bias, void *y, void *workspace, void *stream,
+                              int32_t parts);
+
 /* Size of the device array that ct_run_noalloc uses as its workspace.  Every
  * GPU that loads libct.so holds this much device memory until the process
  * exits. */
@@ -191,13 +216,18 @@ CT_API ct_status ct_run(const ct_plan_t *plan, const void *x, const void *w_pack
  * have no counterpart of this call; it exists only for such callers.  The
  * caller still passes x, w_packed, bias and y as for ct_run.  The workspace
  * comes from a fixed array of CT_NOALLOC_SCRATCH_BYTES inside the library:
- * plans whose ct_workspace_bytes exceed that return CT_ERR_WORKSPACE.  The
- * first call on a device that needs the array looks up its device address on
- * the current device; make that first call before any stream capture.  No
- * call allocates device memory.  All calls share the one array (it keeps the
- * last call's contents; the kernels overwrite all workspace bytes they read),
- * so calls whose GPU work overlaps in time, for example on two streams,
- * race on it and must be serialised by the caller. */
+ * plans whose ct_workspace_bytes exceed that return CT_ERR_WORKSPACE.  Every
+ * call looks up the array's device address on the current device
+ * (cudaGetSymbolAddress; host code only ever sees a stand-in for the array,
+ * never its device address).  With CUDA's lazy module loading the first such
+ * lookup on a device loads the module that holds the array, which takes
+ * CT_NOALLOC_SCRATCH_BYTES of device memory at that moment: make the first
+ * call on each device at start-up, before any stream capture and before the
+ * caller hands the rest of the device memory to its own allocator.  Later
+ * calls allocate nothing.  All calls share the one array (it keeps the last
+ * call's contents; the kernels overwrite all workspace bytes they read), so
+ * calls whose GPU work overlaps in time, for example on two streams, race on
+ * it and must be serialised by the caller. */
 CT_API ct_status ct_run_noalloc(const ct_plan_t *plan, const void *x, const void *w_packed,
                                 const void *bias, void *y, void *stream);
 
@@ -214,10 +244,22 @@ CT_API const char *ct_status_string(ct_status status);
  * earlier on other streams must be finished by the caller), then reads and
  * clears the error words of the current device.  *code = 0 and CT_OK when no
  * wait ran out since the last call; otherwise *code = 100 * module + wait
- * site (module 1 dense_tc, 2 dense_tc_pair, 3 dense_tc_pertap, 4 grouped)
- * and CT_ERR_DEVICE.  CT_ERR_DEVICE with *code = 0 means a CUDA call failed
- * (or the current device is not an sm_100 part). */
+ * site (module 1 dense_tc, 2 dense_tc_pair, 3 dense_tc_pertap, 4 grouped,
+ * 5 the self-test below) and CT_ERR_DEVICE.  CT_ERR_DEVICE with *code = 0
+ * means a CUDA call failed (or the current device is not an sm_100 part). */
 CT_API ct_status ct_take_device_error(void *stream, int32_t *code);
+
+/* Self-test of the bounded-wait failure path (no counterpart on the pages).
+ * One block of one thread runs the steps every tensor-core kernel takes when
+ * a wait runs out: it starts a bulk copy of 4 KB into its shared memory,
+ * then waits, with a limit of `limit_cycles` SM clock cycles (1 .. 2^31),
+ * on an mbarrier that nothing ever arrives at.  When the limit runs out it
+ * records wait site 1 in module 5's error word, waits (with the kernels'
+ * usual one-second limit) for its copy still in flight, and returns.  So
+ * after a call, ct_take_device_error reports code 501 and the device stays
+ * usable; site 2 would mean the copy never completed.  Asynchronous on
+ * `stream`; CT_ERR_ATTR for a limit outside the range. */
+CT_API ct_status ct_selftest_wait_timeout(void *stream, int64_t limit_cycles);
 
 #ifdef __cplusplus
 }

@@ -187,8 +187,27 @@ def test_run_argument_checks_without_device():
         with pytest.raises(ct.CtError) as e:   # fp32 y at an odd address
             ct.ct_run(plan, P(4096), P(4096), P(4096), P(4097), P(0), P(0))
         assert e.value.status == 5
+        # ct_run_parts: the same checks; an unknown part bit is an attribute
+        # error, an empty mask launches nothing
+        with pytest.raises(ct.CtError) as e:
+            ct.ct_run_parts(plan, P(4096), P(4096), P(4096), P(0), P(0), P(0), ct.PART_MAIN)
+        assert e.value.status == 6
+        with pytest.raises(ct.CtError) as e:
+            ct.ct_run_parts(plan, P(4096), P(4096), P(4096), P(4096), P(0), P(0), 4)
+        assert e.value.status == 4
+        ct.ct_run_parts(plan, P(4096), P(4096), P(4096), P(4096), P(0), P(0), 0)
     finally:
         ct.ct_plan_destroy(plan)
+
+
+def test_selftest_argument_checks_without_device():
+    """The bounded-wait self-test refuses a limit outside 1 .. 2^31 before
+    touching a device, and reports CT_ERR_DEVICE when there is none."""
+    L = ct.lib()
+    assert L.ct_selftest_wait_timeout(None, 0) == 4
+    assert L.ct_selftest_wait_timeout(None, (1 << 31) + 1) == 4
+    if not torch.cuda.is_available():
+        assert L.ct_selftest_wait_timeout(None, 1000) == 7
 
 
 def _kernel_for(x_shape, w_shape, dtype, layout="nchw", strides=None, pads=None, group=1):

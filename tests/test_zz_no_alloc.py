@@ -1,15 +1,20 @@
 """ct_run_noalloc against ct_run, on the GPU.
 
-ct_run_noalloc serves callers that may not allocate device memory while they
-run (for example a plugin inside an engine that owns all device memory): it
-takes its workspace from a fixed array inside libct.so instead of from the
-caller.  Here it runs a plan that needs a workspace (fp16 channels-first on
-the tensor-core path, whose input is re-laid channels-last into it) twice in
-a row, on two different inputs, and each result must match what ct_run gives
-with a torch-allocated workspace, within the fp16 parity tolerance.
+ct_run_noalloc serves callers that must not allocate device memory while
+they run, for example a plugin inside an inference engine that owns all of
+the device's memory and hands out only its own buffers.  Such a caller
+still passes X, the packed weight, the bias and Y; the workspace comes from
+a fixed array inside libct.so instead of from the caller.
+
+Here a plan that needs a workspace (fp16 channels-first on the tensor-core
+path, whose input is re-laid channels-last into it) runs twice in a row, on
+two different inputs.  Each result must equal, bit for bit, what ct_run
+gives with a torch-allocated workspace (the same kernels on the same
+inputs), hence also lie within the fp16 parity tolerance of the oracle.  The
+second call must not change the device's free memory.
 
 This file sorts last so that a run that stops at the first failure has
-already run every other test.
+already run every other test; it also passes when run alone.
 """
 
 import numpy as np
@@ -37,19 +42,28 @@ def test_run_noalloc_matches_run_twice():
     assert ct.ct_workspace_bytes(op.plan) <= 32 * 1024 * 1024
     stream = ct._stream_ptr(None)
     rel, ab = TOL[torch.float16]
-    for call, seed in enumerate((503, 504)):
-        x = draw(case["x_shape"], ("normal", 1.0), seed, torch.float16)
-        xd = x.cuda()
-        y_ref = op(xd)                                    # ct_run, torch workspace
-        y = torch.full(op.y_shape, float("nan"), dtype=torch.float16, device="cuda")
-        ct.ct_run_noalloc(op.plan, ct._ptr(xd), ct._ptr(op.w_packed), ct._ptr(op.bias),
-                          ct._ptr(y), stream)
+    xs = [draw(case["x_shape"], ("normal", 1.0), seed, torch.float16) for seed in (503, 504)]
+    xds = [x.cuda() for x in xs]
+    refs = [op(xd) for xd in xds]                         # ct_run, torch workspace
+    ys = [torch.full(op.y_shape, float("nan"), dtype=torch.float16, device="cuda")
+          for _ in xs]
+    torch.cuda.synchronize()
+    free = []
+    for call in range(2):
+        free.append(torch.cuda.mem_get_info()[0])
+        ct.ct_run_noalloc(op.plan, ct._ptr(xds[call]), ct._ptr(op.w_packed), ct._ptr(op.bias),
+                          ct._ptr(ys[call]), stream)
         torch.cuda.synchronize()
-        xa, wa, ba = to_oracle(x, w, b, "nchw")
-        _, absacc = conv_transpose_ref(xa, wa, ba, attrs_from(case))
-        diff = (y.double() - y_ref.double()).abs().cpu().numpy()
-        bound = rel * absacc + ab
-        assert np.all(diff <= bound), "call %d: ct_run_noalloc differs from ct_run" % call
+    free.append(torch.cuda.mem_get_info()[0])
+    # the first call may load the module that holds the array; the second
+    # call allocates nothing
+    assert free[2] == free[1], free
+    for call in range(2):
+        assert torch.equal(ys[call], refs[call]), "call %d: ct_run_noalloc differs from ct_run" % call
+        xa, wa, ba = to_oracle(xs[call], w, b, "nchw")
+        ref, absacc = conv_transpose_ref(xa, wa, ba, attrs_from(case))
+        err = np.abs(ys[call].double().cpu().numpy() - ref)
+        assert np.all(err <= rel * absacc + ab), "call %d: outside the fp16 tolerance" % call
 
 
 def test_run_noalloc_rejects_oversized_workspace():

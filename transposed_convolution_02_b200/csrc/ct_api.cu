@@ -352,7 +352,14 @@ ct_status ct_prepack_weights(const ct_plan_t *plan, const void *w, void *w_packe
 
 ct_status ct_run(const ct_plan_t *plan, const void *x, const void *w_packed, const void *bias,
                  void *y, void *workspace, void *stream) {
+    return ct_run_parts(plan, x, w_packed, bias, y, workspace, stream, CT_PART_ALL);
+}
+
+ct_status ct_run_parts(const ct_plan_t *plan, const void *x, const void *w_packed, const void *bias,
+                       void *y, void *workspace, void *stream, int32_t parts) {
     if (!plan) return CT_ERR_NULL;
+    if (parts & ~CT_PART_ALL) return CT_ERR_ATTR;
+    if (parts == 0) return CT_OK;
     const Plan &p = *reinterpret_cast<const Plan *>(plan);
     const int64_t ny = p.N * p.M * numel_out(p);
     if (ny == 0) return CT_OK;   // empty output: nothing to write
@@ -373,12 +380,13 @@ ct_status ct_run(const ct_plan_t *plan, const void *x, const void *w_packed, con
     if (st != CT_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     switch (p.algo) {
-        case CT_ALGO_DENSE_TC: return dense_tc_run(p, x, w_packed, bias, y, workspace, s);
-        case CT_ALGO_DENSE_TC_PERTAP: return dense_pertap_run(p, x, w_packed, bias, y, workspace, s);
-        case CT_ALGO_DENSE_TC_PAIR: return dense_pair_run(p, x, w_packed, bias, y, workspace, s);
-        case CT_ALGO_GROUPED: return grouped_run(p, x, w_packed, bias, y, s);
-        case CT_ALGO_FP32_GEMM: return fp32_gemm_run(p, x, w_packed, bias, y, s);
-        default: return generic_run(p, x, w_packed, bias, y, s);
+        case CT_ALGO_DENSE_TC: return dense_tc_run(p, x, w_packed, bias, y, workspace, s, parts);
+        case CT_ALGO_DENSE_TC_PERTAP: return dense_pertap_run(p, x, w_packed, bias, y, workspace, s, parts);
+        case CT_ALGO_DENSE_TC_PAIR: return dense_pair_run(p, x, w_packed, bias, y, workspace, s, parts);
+        case CT_ALGO_FP32_GEMM: return fp32_gemm_run(p, x, w_packed, bias, y, s, parts);
+        // one launch: the whole call is its main kernel
+        case CT_ALGO_GROUPED: return (parts & CT_PART_MAIN) ? grouped_run(p, x, w_packed, bias, y, s) : CT_OK;
+        default: return (parts & CT_PART_MAIN) ? generic_run(p, x, w_packed, bias, y, s) : CT_OK;
     }
 }
 
@@ -388,11 +396,11 @@ ct_status ct_take_device_error(void *stream, int32_t *code) {
     ct_status st = check_device();
     if (st != CT_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    // module numbers 1..4: dense_tc, dense_tc_pair, dense_tc_pertap, grouped
-    const int words[4] = {dense_tc_take_error(s), dense_pair_take_error(s), dense_pertap_take_error(s),
-                          grouped_take_error(s)};
+    // module numbers 1..5: dense_tc, dense_tc_pair, dense_tc_pertap, grouped, the self-test
+    const int words[5] = {dense_tc_take_error(s), dense_pair_take_error(s), dense_pertap_take_error(s),
+                          grouped_take_error(s), selftest_take_error(s)};
     bool cuda_failed = false;
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 5; ++i) {
         if (words[i] < 0) cuda_failed = true;
         if (words[i] > 0 && *code == 0) *code = (i + 1) * 100 + words[i];
     }

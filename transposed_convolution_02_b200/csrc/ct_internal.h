@@ -69,7 +69,7 @@ size_t dense_pertap_ws_bytes(const Plan &p);
 void dense_pertap_setup(Plan &p);
 ct_status dense_pertap_prepack(const Plan &p, const void *w, void *wp, cudaStream_t st);
 ct_status dense_pertap_run(const Plan &p, const void *x, const void *wp, const void *bias, void *y,
-                           void *ws, cudaStream_t st);
+                           void *ws, cudaStream_t st, int parts);
 
 bool dense_tc_supports(const Plan &p);
 size_t dense_tc_packed_bytes(const Plan &p);
@@ -77,7 +77,7 @@ size_t dense_tc_ws_bytes(const Plan &p);
 void dense_tc_setup(Plan &p);
 ct_status dense_tc_prepack(const Plan &p, const void *w, void *wp, cudaStream_t st);
 ct_status dense_tc_run(const Plan &p, const void *x, const void *wp, const void *bias, void *y,
-                       void *ws, cudaStream_t st);
+                       void *ws, cudaStream_t st, int parts);
 
 bool dense_pair_supports(const Plan &p);
 bool dense_pair_preferred(const Plan &p);   // auto selection: where it measured fastest
@@ -86,14 +86,14 @@ size_t dense_pair_ws_bytes(const Plan &p);
 void dense_pair_setup(Plan &p);
 ct_status dense_pair_prepack(const Plan &p, const void *w, void *wp, cudaStream_t st);
 ct_status dense_pair_run(const Plan &p, const void *x, const void *wp, const void *bias, void *y,
-                         void *ws, cudaStream_t st);
+                         void *ws, cudaStream_t st, int parts);
 
 bool fp32_gemm_supports(const Plan &p);
 void fp32_gemm_plan(Plan &p);
 size_t fp32_gemm_packed_bytes(const Plan &p);
 ct_status fp32_gemm_prepack(const Plan &p, const void *w, void *wp, cudaStream_t st);
 ct_status fp32_gemm_run(const Plan &p, const void *x, const void *wp, const void *bias, void *y,
-                        cudaStream_t st);
+                        cudaStream_t st, int parts);
 
 bool grouped_supports(const Plan &p);
 void grouped_plan(Plan &p);
@@ -109,6 +109,7 @@ int dense_tc_take_error(cudaStream_t st);
 int dense_pertap_take_error(cudaStream_t st);
 int dense_pair_take_error(cudaStream_t st);
 int grouped_take_error(cudaStream_t st);
+int selftest_take_error(cudaStream_t st);
 
 // Map the last CUDA error to a status (and clear it).
 inline ct_status launch_status() {

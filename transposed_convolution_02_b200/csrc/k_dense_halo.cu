@@ -824,14 +824,16 @@ ct_status dense_tc_prepack(const Plan &p, const void *w, void *wp, cudaStream_t 
 }
 
 ct_status dense_tc_run(const Plan &p, const void *x, const void *wp, const void *bias, void *y,
-                       void *ws, cudaStream_t st) {
+                       void *ws, cudaStream_t st, int parts) {
     const HaloTables &T = tables(p);
     EncodeTiledFn enc = encode_fn();
     if (!enc) return CT_ERR_DEVICE;
     const void *xa = x;
     if (p.layout == CT_NCHW) {
-        ct_status s1 = launch_nchw_to_nhwc_f16(p, x, ws, st);
-        if (s1 != CT_OK) return s1;
+        if (parts & CT_PART_PREPARE) {
+            ct_status s1 = launch_nchw_to_nhwc_f16(p, x, ws, st);
+            if (s1 != CT_OK) return s1;
+        }
         xa = ws;
     }
     CUtensorMap tmA, tmB;
@@ -858,10 +860,11 @@ ct_status dense_tc_run(const Plan &p, const void *x, const void *wp, const void 
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return CT_ERR_DEVICE;
     }
-    if (T.dead) {
+    if (T.dead && (parts & CT_PART_PREPARE)) {
         ct_status s2 = launch_dead_fill(p, bias, y, st);
         if (s2 != CT_OK) return s2;
     }
+    if (!(parts & CT_PART_MAIN)) return CT_OK;
     int grid = sm_count();
     if (grid > T.n_units) grid = T.n_units;
     // programmatic dependent launch: the set-up overlaps the tail of the grid

@@ -1225,11 +1225,11 @@ ct_status dense_pair_prepack(const Plan &p, const void *w, void *wp, cudaStream_
 }
 
 ct_status dense_pair_run(const Plan &p, const void *x, const void *wp, const void *bias, void *y, void *ws,
-                         cudaStream_t st) {
+                         cudaStream_t st, int parts) {
     const PairTables &T = ptables(p);
     EncodeTiledFn enc = encode_fn();
     if (!enc) return CT_ERR_DEVICE;
-    {
+    if (parts & CT_PART_PREPARE) {
         const long long S = (long long)T.in[0] * T.in[1] * T.in[2];
         const long long tiles = ceil_div(S, kPadS);
         PadGeo g;
@@ -1301,10 +1301,11 @@ ct_status dense_pair_run(const Plan &p, const void *x, const void *wp, const voi
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return CT_ERR_DEVICE;
     }
-    if (T.dead) {
+    if (T.dead && (parts & CT_PART_PREPARE)) {
         ct_status s2 = launch_dead_fill(p, bias, y, st);
         if (s2 != CT_OK) return s2;
     }
+    if (!(parts & CT_PART_MAIN)) return CT_OK;
     if (T.f32) {
         if (T.act == CT_ACT_RELU) return launch_pair<CT_ACT_RELU, float>(T, tmA, tmB, tmBs, bias, y, st);
         return launch_pair<CT_ACT_IDENTITY, float>(T, tmA, tmB, tmBs, bias, y, st);

@@ -446,14 +446,16 @@ ct_status dense_pertap_prepack(const Plan &p, const void *w, void *wp, cudaStrea
 }
 
 ct_status dense_pertap_run(const Plan &p, const void *x, const void *wp, const void *bias, void *y,
-                       void *ws, cudaStream_t st) {
+                       void *ws, cudaStream_t st, int parts) {
     const DenseTables &T = tables(p);
     EncodeTiledFn enc = encode_fn();
     if (!enc) return CT_ERR_DEVICE;
     const void *xa = x;
     if (p.layout == CT_NCHW) {
-        ct_status s1 = launch_nchw_to_nhwc_f16(p, x, ws, st);
-        if (s1 != CT_OK) return s1;
+        if (parts & CT_PART_PREPARE) {
+            ct_status s1 = launch_nchw_to_nhwc_f16(p, x, ws, st);
+            if (s1 != CT_OK) return s1;
+        }
         xa = ws;
     }
     CUtensorMap tmA, tmB;
@@ -481,10 +483,11 @@ ct_status dense_pertap_run(const Plan &p, const void *x, const void *wp, const v
                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return CT_ERR_DEVICE;
     }
-    if (T.dead) {
+    if (T.dead && (parts & CT_PART_PREPARE)) {
         ct_status s2 = launch_dead_fill(p, bias, y, st);
         if (s2 != CT_OK) return s2;
     }
+    if (!(parts & CT_PART_MAIN)) return CT_OK;
     const size_t sm = smem_bytes(T);
     static std::atomic<int> attr_set[64];
     if (!allow_smem(dense_pertap_kernel, attr_set, 227 * 1024)) return CT_ERR_DEVICE;

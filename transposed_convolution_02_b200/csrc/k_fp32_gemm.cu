@@ -327,9 +327,9 @@ ct_status fp32_gemm_prepack(const Plan &p, const void *w, void *wp, cudaStream_t
 }
 
 ct_status fp32_gemm_run(const Plan &p, const void *x, const void *wp, const void *bias, void *y,
-                        cudaStream_t st) {
+                        cudaStream_t st, int parts) {
     const F32Args &A = fargs(p);
-    if (has_dead_phases(p)) {
+    if (has_dead_phases(p) && (parts & CT_PART_PREPARE)) {
         uint64_t lm[3] = {0, 0, 0};
         for (int a = 0; a < 3; ++a)
             for (int r = 0; r < p.s[a] && r < 64; ++r)
@@ -342,6 +342,7 @@ ct_status fp32_gemm_run(const Plan &p, const void *x, const void *wp, const void
         ct_status s1 = launch_status();
         if (s1 != CT_OK) return s1;
     }
+    if (!(parts & CT_PART_MAIN)) return CT_OK;
     const long long grid = (long long)A.n_phases * A.tiles_m * A.tiles_p * A.N;
     fp32_gemm_kernel<<<(unsigned)grid, 256, 0, st>>>(A, (const float *)x, (const float *)wp, (const float *)bias,
                                                     (float *)y);

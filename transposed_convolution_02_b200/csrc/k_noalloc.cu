@@ -8,24 +8,22 @@
 // the workspace from a fixed array compiled into the library.
 //
 // The array is a file-scope __device__ variable, so every GPU that loads the
-// library holds CT_NOALLOC_SCRATCH_BYTES of it until the process exits.  Its
-// device address is looked up once per device (cudaGetSymbolAddress, with that
-// device current) on the first call that needs it; host code must never hand
-// the symbol itself to a kernel, since on the host it only names a stand-in.
-// All calls share the one array and it keeps the last call's contents: the
-// kernels overwrite every workspace byte they later read, so nothing needs
-// clearing, but calls whose GPU work overlaps (different streams) race on it.
-#include <mutex>
-
+// library's device code holds CT_NOALLOC_SCRATCH_BYTES of it until the
+// process exits.  Host code never hands the symbol itself to a kernel (on the
+// host it only names a stand-in): every call looks up the array's device
+// address with cudaGetSymbolAddress on the current device, which allocates
+// nothing once the module is loaded and stays right after a device reset.
+// With lazy module loading the first lookup on a device loads the module, and
+// with it the array; callers make that first call at start-up.  All calls
+// share the one array and it keeps the last call's contents: the kernels
+// overwrite every workspace byte they later read, so nothing needs clearing,
+// but calls whose GPU work overlaps (different streams) race on it.
 #include "ct_cuda_util.h"
 #include "ct_internal.h"
 
 namespace {
 
 static __device__ __align__(256) unsigned char g_ct_noalloc_scratch[CT_NOALLOC_SCRATCH_BYTES];
-
-std::mutex g_scratch_mu;
-void *g_scratch_ptr[64];
 
 }  // namespace
 
@@ -38,18 +36,11 @@ extern "C" ct_status ct_run_noalloc(const ct_plan_t *plan, const void *x, const 
     if (need > (size_t)CT_NOALLOC_SCRATCH_BYTES) return CT_ERR_WORKSPACE;
     void *ws = nullptr;
     if (need > 0) {
-        const int dev = ct::current_device();
-        if (dev < 0 || dev >= 64) return CT_ERR_DEVICE;
-        std::lock_guard<std::mutex> lock(g_scratch_mu);
-        if (!g_scratch_ptr[dev]) {
-            void *p = nullptr;
-            if (cudaGetSymbolAddress(&p, g_ct_noalloc_scratch) != cudaSuccess || !p) {
-                cudaGetLastError();
-                return CT_ERR_DEVICE;
-            }
-            g_scratch_ptr[dev] = p;
+        if (ct::current_device() < 0) return CT_ERR_DEVICE;
+        if (cudaGetSymbolAddress(&ws, g_ct_noalloc_scratch) != cudaSuccess || !ws) {
+            cudaGetLastError();
+            return CT_ERR_DEVICE;
         }
-        ws = g_scratch_ptr[dev];
     }
     return ct_run(plan, x, w_packed, bias, y, ws, stream);
 }

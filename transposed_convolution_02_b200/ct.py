@@ -30,10 +30,13 @@ AUTOPAD = {"NOTSET": 0, "SAME_UPPER": 1, "SAME_LOWER": 2, "VALID": 3}
 ALGO = {"auto": 0, "generic": 1, "dense_tc": 2, "fp32_gemm": 3, "grouped": 4,
         "dense_tc_pertap": 5, "dense_tc_pair": 6}
 
+PART_PREPARE, PART_MAIN, PART_ALL = 1, 2, 3
+
 EXPORTED = ["ct_output_shape", "ct_plan", "ct_plan_kernel", "ct_plan_launches",
             "ct_prepacked_weight_bytes",
-            "ct_workspace_bytes", "ct_prepack_weights", "ct_run", "ct_run_noalloc",
-            "ct_plan_destroy", "ct_status_string", "ct_take_device_error"]
+            "ct_workspace_bytes", "ct_prepack_weights", "ct_run", "ct_run_parts",
+            "ct_run_noalloc", "ct_plan_destroy", "ct_status_string", "ct_take_device_error",
+            "ct_selftest_wait_timeout"]
 
 
 class CtError(RuntimeError):
@@ -80,6 +83,8 @@ def lib():
         L.ct_workspace_bytes.argtypes = [P, szp]
         L.ct_prepack_weights.argtypes = [P, P, P, P]
         L.ct_run.argtypes = [P, P, P, P, P, P, P]
+        L.ct_run_parts.argtypes = [P, P, P, P, P, P, P, ctypes.c_int32]
+        L.ct_selftest_wait_timeout.argtypes = [P, ctypes.c_int64]
         L.ct_run_noalloc.argtypes = [P, P, P, P, P, P]
         L.ct_plan_destroy.argtypes = [P]
         L.ct_plan_destroy.restype = None
@@ -87,8 +92,8 @@ def lib():
         L.ct_status_string.argtypes = [ctypes.c_int]
         L.ct_status_string.restype = ctypes.c_char_p
         for name in ("ct_output_shape", "ct_plan", "ct_plan_launches", "ct_prepacked_weight_bytes",
-                     "ct_workspace_bytes", "ct_prepack_weights", "ct_run", "ct_run_noalloc",
-                     "ct_take_device_error"):
+                     "ct_workspace_bytes", "ct_prepack_weights", "ct_run", "ct_run_parts",
+                     "ct_run_noalloc", "ct_take_device_error", "ct_selftest_wait_timeout"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -157,6 +162,23 @@ def ct_run(plan, x_ptr, wp_ptr, bias_ptr, y_ptr, ws_ptr, stream):
     st = lib().ct_run(plan, x_ptr, wp_ptr, bias_ptr, y_ptr, ws_ptr, stream)
     if st != CT_OK:
         raise CtError(st, "ct_run")
+
+
+def ct_run_parts(plan, x_ptr, wp_ptr, bias_ptr, y_ptr, ws_ptr, stream, parts):
+    """ct_run restricted to a mask of PART_PREPARE (re-layout, bias fill) and
+    PART_MAIN (the main kernel), for timing the parts of a call apart."""
+    st = lib().ct_run_parts(plan, x_ptr, wp_ptr, bias_ptr, y_ptr, ws_ptr, stream, int(parts))
+    if st != CT_OK:
+        raise CtError(st, "ct_run_parts")
+
+
+def ct_selftest_wait_timeout(limit_cycles, stream=None):
+    """Launch the bounded-wait self-test (a wait that gives up after
+    `limit_cycles` SM cycles, then drains its copy in flight); the next
+    ct_take_device_error() returns 501."""
+    st = lib().ct_selftest_wait_timeout(_stream_ptr(stream), int(limit_cycles))
+    if st != CT_OK:
+        raise CtError(st, "ct_selftest_wait_timeout")
 
 
 def ct_run_noalloc(plan, x_ptr, wp_ptr, bias_ptr, y_ptr, stream):
@@ -308,11 +330,21 @@ class ConvTranspose:
                _ptr(self.workspace), _stream_ptr(stream))
         return y
 
-    def run_ptrs(self, x_ptr, y_ptr, stream_ptr):
+    def run_ptrs(self, x_ptr, y_ptr, stream_ptr, parts=PART_ALL):
         """Launch on raw device pointers (benchmark loops); the caller
-        guarantees buffers of the planned shapes, dtype and device."""
-        ct_run(self.plan, x_ptr, _ptr(self.w_packed), _ptr(self.bias), y_ptr,
-               _ptr(self.workspace), stream_ptr)
+        guarantees buffers of the planned shapes, dtype and device.  `parts`
+        restricts the call to its preparation or main launches."""
+        ct_run_parts(self.plan, x_ptr, _ptr(self.w_packed), _ptr(self.bias), y_ptr,
+                     _ptr(self.workspace), stream_ptr, parts)
+
+    def run_part(self, x, out, parts, stream=None):
+        """ct_run_parts on tensors checked against the plan (see run_ptrs)."""
+        check_io(x, out, self.x_shape, self.y_shape, self.dtype, self.device)
+        if out is None or not x.is_contiguous():
+            raise ValueError("run_part needs a contiguous X and an out tensor")
+        ct_run_parts(self.plan, _ptr(x), _ptr(self.w_packed), _ptr(self.bias), _ptr(out),
+                     _ptr(self.workspace), _stream_ptr(stream), parts)
+        return out
 
     def __del__(self):
         try:
