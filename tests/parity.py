@@ -105,6 +105,60 @@ def sampled_points(y_shape_cf, rng, n_random=1500):
     return np.array(sorted(pts), dtype=np.int64)
 
 
+def stratified_points(y_shape_cf, strides, rng, chunk=16, mblock=32):
+    """Output points (n, m, o..) in channels-first coordinates that reach every
+    piece of work a kernel can own.  For every image n, every stride phase r
+    (o mod s per axis), every block of `mblock` output channels and every run
+    of `chunk` consecutive positions J of the phase (J numbered with the last
+    axis fastest), one random point; plus the first and the last J of every
+    row of every phase (row ends and tile edges).  A unit, CTA, warp or lane
+    group that owns at least `chunk` consecutive positions of a phase row, or
+    whole rows, for one block of channels therefore gets a point."""
+    dims = [int(d) for d in y_shape_cf]
+    n_img, m_all, out = dims[0], dims[1], dims[2:]
+    r = len(out)
+    s = [int(v) for v in strides]
+    pts = []
+    for ph in np.ndindex(*s):
+        nj = [(out[a] - ph[a] + s[a] - 1) // s[a] if out[a] > ph[a] else 0 for a in range(r)]
+        total = int(np.prod(nj))
+        if total == 0:
+            continue
+        starts = np.arange(0, total, chunk)
+        width = np.minimum(chunk, total - starts)
+        mstarts = np.arange(0, m_all, mblock)
+        mwidth = np.minimum(mblock, m_all - mstarts)
+        for n in range(n_img):
+            t = starts[:, None] + (rng.random((len(starts), len(mstarts))) * width[:, None]).astype(np.int64)
+            m = mstarts[None, :] + (rng.random((len(starts), len(mstarts))) * mwidth[None, :]).astype(np.int64)
+            t, m = t.reshape(-1), m.reshape(-1)
+            J = np.stack(np.unravel_index(t, nj), axis=1)
+            o = J * np.array(s)[None, :] + np.array(ph)[None, :]
+            pts.append(np.concatenate([np.full((len(t), 1), n), m[:, None], o], axis=1))
+            # both ends of every row of the phase
+            rows = int(np.prod(nj[:-1]))
+            for jx in {0, nj[-1] - 1}:
+                rj = np.stack(np.unravel_index(np.arange(rows), nj[:-1]), axis=1) if r > 1 else \
+                    np.zeros((1, 0), dtype=np.int64)
+                J = np.concatenate([rj, np.full((rows, 1), jx)], axis=1)
+                o = J * np.array(s)[None, :] + np.array(ph)[None, :]
+                m = rng.integers(0, m_all, rows)
+                pts.append(np.concatenate([np.full((rows, 1), n), m[:, None], o], axis=1))
+    allp = np.concatenate(pts, axis=0).astype(np.int64)
+    return np.unique(allp, axis=0)
+
+
+def check_points(op, y, x, w, b, case, dtype, layout, pts, where):
+    """Compare the GPU output at `pts` (channels-first coordinates) with the
+    oracle evaluated at those points one by one."""
+    xa, wa, ba = to_oracle(x, w, b, layout)
+    ycf = y if layout == "nchw" else y.movedim(-1, 1)
+    ref, absacc = conv_transpose_points(xa, wa, ba, attrs_from(case), pts,
+                                        activation=case.get("activation", "identity"))
+    got = ycf[tuple(torch.from_numpy(pts.T).to(y.device))].double().cpu().numpy()
+    return check_close(got, ref, absacc, dtype, where)
+
+
 def sampled_parity(op, y, x, w, b, case, dtype, layout, rng, n_random=1500):
     """Compare the full GPU output with oracle points one by one."""
     xa, wa, ba = to_oracle(x, w, b, layout)

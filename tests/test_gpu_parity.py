@@ -11,8 +11,8 @@ import pytest
 import torch
 
 from cases import random_case
-from parity import (check_close, draw_case, full_parity, gpu_run, sampled_parity, to_oracle,
-                    attrs_from)
+from parity import (check_close, check_points, draw_case, full_parity, gpu_run, sampled_parity,
+                    stratified_points, to_oracle, attrs_from)
 from oracle import conv_transpose_ref
 from transposed_convolution_02_b200 import ct
 from transposed_convolution_02_b200.workloads import WORKLOADS, make_inputs
@@ -59,31 +59,40 @@ def test_generic_empty_and_degenerate():
     assert y.shape == (0, 2, 11)
 
 
+# Kernel that automatic selection must pick for each reduced workload, per
+# layout (sizes above the 1e7-FLOP threshold under which the gather kernel is
+# chosen, so each reduced case runs on the kernel family of its workload).
+REDUCED = {
+    1: ([1, 8, 8, 8], [8, 4, 3, 3], None, ("generic", "generic")),
+    2: ([2, 96, 13, 21], [96, 40, 4, 4], None, ("dense_tc_pair", "dense_tc")),
+    3: ([1, 64, 6, 8, 10], [64, 32, 3, 3, 3], None, ("dense_tc", "dense_tc")),
+    4: ([2, 72, 45], [72, 52, 16], None, ("dense_tc_pair", "dense_tc_pair")),
+    5: ([2, 128, 12, 14], [128, 16, 3, 3], 8, ("grouped", "generic")),
+}
+
+
 @pytest.mark.parametrize("wid", [1, 2, 3, 4, 5])
 def test_workload_reduced(wid):
-    """Each workload's attributes on reduced sizes, whole output compared."""
+    """Each workload's attributes on reduced sizes, whole output compared, on
+    the kernel automatic selection picks for the workload's family."""
     wl = WORKLOADS[wid]
     case = _wl_case(wl)
-    x_shape = list(wl.x_shape)
-    w_shape = list(wl.w_shape)
-    if wid == 2:
-        x_shape, w_shape = [2, 96, 13, 21], [96, 40, 4, 4]
-    elif wid == 3:
-        x_shape, w_shape = [1, 24, 5, 6, 7], [24, 20, 3, 3, 3]
-    elif wid == 4:
-        x_shape, w_shape = [2, 72, 45], [72, 52, 16]
-    elif wid == 5:
-        x_shape, w_shape = [2, 64, 9, 11], [64, 16, 3, 3]
-        case["group"] = 4
-    case["x_shape"], case["w_shape"] = x_shape, w_shape
-    for layout in ("nchw", "nhwc"):
-        full_parity(case, wl.dtype, 900 + wid, layout)
+    x_shape, w_shape, group, kernels = REDUCED[wid]
+    case["x_shape"], case["w_shape"] = list(x_shape), list(w_shape)
+    if group is not None:
+        case["group"] = group
+    for layout, kernel in zip(("nchw", "nhwc"), kernels):
+        full_parity(case, wl.dtype, 900 + wid, layout, expect_kernel=kernel)
 
 
 @pytest.mark.parametrize("wid", [1, 2, 3, 4, 5])
 def test_workload_full_size(wid):
     """The workload at full size, auto-chosen kernel (the launch the benchmark
-    times): sampled outputs against the oracle, plus whole-output properties."""
+    times): stratified and random outputs against the oracle evaluated point
+    by point, plus whole-output properties.  The stratified set holds a point
+    for every (image, stride phase, 32-channel block, run of 16 consecutive
+    positions of the phase) and both ends of every phase row, so every unit,
+    CTA, epilogue warp and channel piece of the kernel is checked."""
     wl = WORKLOADS[wid]
     case = _wl_case(wl)
     x, w, b = make_inputs(wl)
@@ -92,6 +101,9 @@ def test_workload_full_size(wid):
     rng = np.random.default_rng(wid)
     sampled_parity(op, y, x, w, b, case, wl.dtype, "nchw", rng,
                    n_random=400 if wid in (2, 4) else 1500)
+    pts = stratified_points(list(y.shape), wl.strides, rng,
+                            mblock=16 if wl.group > 1 else 32)
+    check_points(op, y, x, w, b, case, wl.dtype, "nchw", pts, "stratified workload %d" % wid)
     if wid == 1:
         xa, wa, ba = to_oracle(x, w, b, "nchw")
         ref, absacc = conv_transpose_ref(xa, wa, ba, attrs_from(case))
@@ -101,6 +113,115 @@ def test_workload_full_size(wid):
         bb = b.cuda().view(1, -1, 1, 1).expand(y.shape[0], -1, y.shape[2], y.shape[3])
         assert torch.equal(y[:, :, 0::2, :], bb[:, :, 0::2, :])
         assert torch.equal(y[:, :, :, 0::2], bb[:, :, :, 0::2])
+
+
+# Attribute paths of the ai.onnx.ConvTranspose README ("Attributes") that the
+# workloads do not exercise, each through the tensor-core and grouped kernels:
+# output_shape (its pads split at the end under NOTSET, like SAME_LOWER under
+# SAME_LOWER), VALID, an explicit kernel_shape, and SAME totals that are
+# negative (kernel 1, stride 2) under both SAME rules.
+ATTR_CASES = [
+    dict(x_shape=[2, 64, 9, 10], w_shape=[64, 48, 4, 4], strides=[2, 2], output_shape=[17, 19],
+         bias=True),
+    dict(x_shape=[2, 64, 9, 10], w_shape=[64, 48, 4, 4], strides=[2, 2], output_shape=[17, 19],
+         auto_pad="SAME_LOWER", bias=True),
+    dict(x_shape=[2, 64, 9, 10], w_shape=[64, 48, 3, 3], strides=[2, 2], auto_pad="VALID",
+         bias=True),
+    dict(x_shape=[2, 64, 9, 10], w_shape=[64, 48, 4, 4], strides=[2, 2], kernel_shape=[4, 4],
+         pads=[1, 2, 0, 1], bias=True),
+    dict(x_shape=[2, 64, 9, 10], w_shape=[64, 48, 1, 1], strides=[2, 2], auto_pad="SAME_LOWER",
+         bias=True),
+    dict(x_shape=[2, 64, 9, 10], w_shape=[64, 48, 1, 1], strides=[2, 2], auto_pad="SAME_UPPER",
+         bias=True),
+    dict(x_shape=[1, 32, 5, 6, 7], w_shape=[32, 24, 3, 3, 3], strides=[2, 2, 2],
+         output_shape=[9, 12, 13], auto_pad="SAME_LOWER", bias=True),
+]
+
+
+@pytest.mark.parametrize("idx", range(len(ATTR_CASES)))
+@pytest.mark.parametrize("algo,dtype,layout", [
+    ("dense_tc_pair", torch.float16, "nchw"),
+    ("dense_tc", torch.float16, "nchw"),
+    ("dense_tc", torch.float16, "nhwc"),
+    ("dense_tc_pair", torch.float32, "nchw"),
+    ("dense_tc_pair", torch.float16, "nhwc"),
+])
+def test_attribute_paths_on_tensor_cores(idx, algo, dtype, layout):
+    case = ATTR_CASES[idx]
+    try:
+        full_parity(case, dtype, 1200 + idx, layout, algo=algo, expect_kernel=algo)
+    except ct.CtError as e:
+        # only a kernel-capability refusal at plan time is acceptable
+        assert e.status == 9, e
+        assert algo == "dense_tc" and len(case["x_shape"]) == 5, (algo, case)
+
+
+@pytest.mark.parametrize("case", [
+    dict(x_shape=[2, 64, 9, 10], w_shape=[64, 16, 3, 3], strides=[2, 2], output_shape=[17, 19],
+         group=4, bias=True),
+    dict(x_shape=[2, 64, 9, 10], w_shape=[64, 16, 3, 3], strides=[2, 2], dilations=[2, 2],
+         output_shape=[19, 21], auto_pad="SAME_LOWER", group=4, bias=True),
+    dict(x_shape=[2, 64, 9, 10], w_shape=[64, 16, 3, 3], strides=[2, 2], auto_pad="VALID",
+         group=4, bias=True),
+    dict(x_shape=[2, 64, 9, 16], w_shape=[64, 16, 1, 1], strides=[2, 2], auto_pad="SAME_LOWER",
+         group=2, bias=True),
+    dict(x_shape=[2, 64, 9, 10], w_shape=[64, 16, 3, 3], strides=[2, 2], kernel_shape=[3, 3],
+         pads=[0, 2, 1, 1], group=4, bias=True),
+])
+def test_attribute_paths_grouped(case):
+    full_parity(case, torch.float16, 1300, "nchw", algo="grouped", expect_kernel="grouped")
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.float32])
+def test_channels_last_wrapper(dtype):
+    """conv_transpose_nhwc in the ClikaRT::ops::conv_transpose form: input
+    [N, D.., C_in], weight [C_in, K.., O/groups], padding as interleaved
+    (lo, hi) pairs per spatial dim, activation; checked against the oracle
+    with the pads split into the README's begins and ends."""
+    rng = np.random.default_rng(17)
+    for i, (xs, ws, st, pad_lohi, op_, g, act) in enumerate([
+        ([2, 64, 9, 10], [64, 48, 4, 4], [2, 2], [1, 2, 0, 1], [0, 0], 1, "identity"),
+        ([2, 64, 9, 10], [64, 48, 3, 3], [2, 2], [2, 0, 1, 1], [1, 1], 1, "relu"),
+        ([2, 32, 300], [32, 24, 16], [8], [3, 5], [0], 1, "identity"),
+        ([1, 32, 5, 6, 7], [32, 16, 3, 3, 3], [2, 2, 2], [1, 1, 0, 2, 1, 0], [1, 0, 1], 1, "relu"),
+        ([2, 64, 7, 9], [64, 8, 3, 3], [2, 2], [1, 0, 0, 1], [0, 0], 4, "identity"),
+    ]):
+        r = len(xs) - 2
+        begins = [pad_lohi[2 * a] for a in range(r)]
+        ends = [pad_lohi[2 * a + 1] for a in range(r)]
+        case = dict(x_shape=xs, w_shape=ws, strides=st, pads=begins + ends, output_padding=op_,
+                    group=g, bias=True, activation=act)
+        x, w, b = draw_case(case, dtype, 1400 + i, "nhwc")
+        y = ct.conv_transpose_nhwc(x.cuda(), w.cuda(), b.cuda(), stride=st, padding=pad_lohi,
+                                   output_padding=op_, groups=g, dilation=[1] * r,
+                                   activation=act)
+        torch.cuda.synchronize()
+        xa, wa, ba = to_oracle(x, w, b, "nhwc")
+        ref, absacc = conv_transpose_ref(xa, wa, ba, attrs_from(case), activation=act)
+        check_close(y, np.moveaxis(ref, 1, -1), np.moveaxis(absacc, 1, -1), dtype,
+                    "conv_transpose_nhwc %d" % i)
+
+
+def test_channels_first_wrapper():
+    """conv_transpose, the one-call channels-first form, on the attribute
+    paths of the README table (output_shape, SAME_LOWER, dilations, group)."""
+    for i, case in enumerate([
+        dict(x_shape=[2, 64, 9, 10], w_shape=[64, 48, 4, 4], strides=[2, 2], output_shape=[17, 19],
+             auto_pad="SAME_LOWER", bias=True),
+        dict(x_shape=[2, 64, 9, 10], w_shape=[64, 16, 3, 3], strides=[2, 2], dilations=[2, 2],
+             auto_pad="SAME_UPPER", group=4, bias=True),
+        dict(x_shape=[2, 36, 200], w_shape=[36, 20, 16], strides=[8], pads=[4, 4], bias=False),
+    ]):
+        dtype = torch.float32 if len(case["x_shape"]) == 3 else torch.float16
+        x, w, b = draw_case(case, dtype, 1500 + i)
+        y = ct.conv_transpose(x.cuda(), w.cuda(), b.cuda() if b is not None else None,
+                              strides=case["strides"], dilations=case.get("dilations"),
+                              pads=case.get("pads"), auto_pad=case.get("auto_pad", "NOTSET"),
+                              group=case.get("group", 1), output_shape=case.get("output_shape"))
+        torch.cuda.synchronize()
+        xa, wa, ba = to_oracle(x, w, b, "nchw")
+        ref, absacc = conv_transpose_ref(xa, wa, ba, attrs_from(case))
+        check_close(y, ref, absacc, dtype, "conv_transpose %d" % i)
 
 
 def _dense_case(rng, lim_in):
@@ -481,3 +602,24 @@ def test_general_shapes_sampled(idx):
     assert op.kernel in ("dense_tc_pair", "dense_tc"), (name, op.kernel)
     assert not torch.isnan(y).any(), name
     sampled_parity(op, y, x, w, b, case, dt, layout, np.random.default_rng(idx), n_random=600)
+
+
+def test_multi_device_batch_split():
+    """MultiDeviceConvTranspose: one caller's batch split into slices, one
+    plan and packed weight per device, Y gathered on the first device.  With
+    one GPU the slices share cuda:0, which still runs the split, the per-slice
+    plans and the gather through the library's kernels."""
+    from transposed_convolution_02_b200.shard import MultiDeviceConvTranspose
+    # (every slice above the 1e7 FLOP under which the gather kernel is chosen)
+    case = dict(x_shape=[5, 64, 16, 20], w_shape=[64, 48, 4, 4], strides=[2, 2],
+                pads=[1, 1, 1, 1], bias=True)
+    x, w, b = draw_case(case, torch.float16, 1600)
+    md = MultiDeviceConvTranspose(w.cuda(), case["x_shape"], b.cuda(), devices=["cuda:0"] * 3,
+                                  strides=case["strides"], pads=case["pads"])
+    assert [op.x_shape[0] for op in md.ops] == [2, 2, 1]
+    assert all(op.kernel == "dense_tc_pair" for op in md.ops)
+    y = md.gather(md(x.cuda()))
+    torch.cuda.synchronize()
+    xa, wa, ba = to_oracle(x, w, b, "nchw")
+    ref, absacc = conv_transpose_ref(xa, wa, ba, attrs_from(case))
+    check_close(y, ref, absacc, torch.float16, "multi-device batch split")
