@@ -89,13 +89,17 @@ def roofline_for(wl, seconds_per_launch, peaks, sms, kernel=None):
                     unit="TFLOP/s", frac=(flop / seconds_per_launch / 1e12) / peak)
     t_tc = flop / (peaks["tc_tflops"] * 1e12)
     t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    # both fractions, whichever bounds: the fp16 targets are stated against
+    # the tensor peak even where HBM is the binding resource
+    both = dict(tensor_frac=flop / seconds_per_launch / 1e12 / peaks["tc_tflops"],
+                hbm_frac=nbytes / seconds_per_launch / 1e9 / peaks["hbm_gbs"])
     if t_tc >= t_hbm:
         a = flop / seconds_per_launch / 1e12
         return dict(bound="tensor", achieved=a, peak=peaks["tc_tflops"], unit="TFLOP/s",
-                    frac=a / peaks["tc_tflops"])
+                    frac=a / peaks["tc_tflops"], **both)
     a = nbytes / seconds_per_launch / 1e9
     return dict(bound="hbm", achieved=a, peak=peaks["hbm_gbs"], unit="GB/s",
-                frac=a / peaks["hbm_gbs"])
+                frac=a / peaks["hbm_gbs"], **both)
 
 
 def profile_record(wid, kernel):
@@ -121,17 +125,26 @@ def traffic_for(wid, kernel):
     return rec["bytes_per_launch"] if rec else None
 
 
-def annotate_roofline(roof, wid, kernel, launches):
-    """Scope of the achieved figure: it is measured over whole calls (all of a
-    call's launches); with the dominant kernel's share of a call from the
-    committed launch list, the kernel-only fraction follows."""
-    roof["traffic"] = traffic_for(wid, kernel)
-    roof["kernel"] = kernel
-    roof["scope"] = "whole call (%d launch%s), CUDA events" % (launches, "" if launches == 1 else "es")
+def annotate_roofline(roof, wid, kernel, launches, call_seconds=None, flop=None, nbytes=None):
+    """Scope and provenance of the roofline figures.  `achieved` and `frac`
+    are the dominant kernel's, timed alone (CUDA events over launches of that
+    kernel only); the whole call (all of its launches) is given beside it.
+    `traffic` is DRAM read + write bytes of one steady-state launch from the
+    committed ncu record, while the kernel source still matches it."""
     rec = profile_record(wid, kernel)
-    if rec and launches > 1 and rec.get("share_of_call"):
-        roof["kernel_share_of_call"] = rec["share_of_call"]
-        roof["kernel_frac_est"] = roof["frac"] / rec["share_of_call"]
+    roof["traffic"] = rec["bytes_per_launch"] if rec else None
+    if rec:
+        roof["traffic_detail"] = {k: rec[k] for k in ("dram_read", "dram_write", "l2_write_from_sm",
+                                                       "capture") if k in rec}
+        if nbytes:
+            roof["traffic_over_algorithmic"] = rec["bytes_per_launch"] / nbytes
+    roof["kernel"] = kernel
+    roof["scope"] = ("dominant kernel alone, CUDA events; the call is %d launch%s"
+                     % (launches, "" if launches == 1 else "es"))
+    if call_seconds is not None:
+        roof["call_us"] = call_seconds * 1e6
+        roof["call_frac"] = roof["frac"] * roof["kernel_us"] / roof["call_us"] \
+            if roof.get("kernel_us") else None
     return roof
 
 
@@ -207,8 +220,35 @@ def build_op(wl, device):
     return op, x
 
 
-def time_device(wl, device, steps, warmup, l2_bytes, dist_max=None, sampler=None):
-    """Device time of `steps` ct_runs (CUDA graphs, rotating buffer sets)."""
+def _graph_set(op, xs, ys, parts):
+    """One CUDA graph per buffer set, each holding one call restricted to `parts`."""
+    graphs = []
+    for i in range(len(xs)):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            op.run_part(xs[i], ys[i], parts)
+        graphs.append(g)
+    return graphs
+
+
+def _replay_ms(graphs, steps, first, sampler=None):
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    ctx = sampler if sampler is not None else _Null()
+    with ctx:
+        start.record()
+        for j in range(steps):
+            graphs[(first + j) % len(graphs)].replay()
+        end.record()
+        torch.cuda.synchronize()
+    return start.elapsed_time(end)
+
+
+def time_device(wl, device, steps, warmup, l2_bytes, dist_max=None, sampler=None, kernel_steps=None):
+    """Device time of `steps` ct_runs (CUDA graphs, rotating buffer sets),
+    then of `kernel_steps` launches of the call's main kernel alone (the
+    preparation launches replayed once before, so its workspace is in place)
+    and of the preparation alone.  Returns (ms for `steps` calls, info)."""
     op, x_cpu = build_op(wl, device)
     xb = x_cpu.numel() * x_cpu.element_size()
     yb = math.prod(op.y_shape) * x_cpu.element_size()
@@ -218,7 +258,6 @@ def time_device(wl, device, steps, warmup, l2_bytes, dist_max=None, sampler=None
         nsets -= 1
     xs = [x_cpu.to(device) for _ in range(nsets)]
     ys = [torch.empty(op.y_shape, dtype=wl.dtype, device=device) for _ in range(nsets)]
-    graphs = []
     s = torch.cuda.Stream(device)
     s.wait_stream(torch.cuda.current_stream(device))
     with torch.cuda.stream(s):
@@ -226,32 +265,57 @@ def time_device(wl, device, steps, warmup, l2_bytes, dist_max=None, sampler=None
             op(xs[i], out=ys[i])
     torch.cuda.current_stream(device).wait_stream(s)
     torch.cuda.synchronize(device)
-    for i in range(nsets):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            op(xs[i], out=ys[i])
-        graphs.append(g)
+    graphs = _graph_set(op, xs, ys, ct.PART_ALL)
     for j in range(warmup):
         graphs[j % nsets].replay()
     if dist_max is not None:
         dist_max("barrier")
     torch.cuda.synchronize(device)
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
-    ctx = sampler if sampler is not None else _Null()
-    with ctx:
-        start.record()
-        for j in range(steps):
-            graphs[(warmup + j) % nsets].replay()
-        end.record()
-        torch.cuda.synchronize(device)
+    ms = _replay_ms(graphs, steps, warmup, sampler)
     if dist_max is not None:
         dist_max("barrier")
-    ms = start.elapsed_time(end)
     info = dict(kernel=op.kernel, launches_per_step=op.launches, sets=nsets,
                 set_bytes=xb + yb)
     del graphs
+    # the main kernel alone, and the preparation alone (rank-local timings:
+    # every rank runs the same steps, no collective in between)
+    ksteps = kernel_steps if kernel_steps is not None else min(steps, 400)
+    main = _graph_set(op, xs, ys, ct.PART_MAIN)
+    for j in range(max(3, warmup // 4)):
+        main[j % nsets].replay()
+    torch.cuda.synchronize(device)
+    info["kernel_ms_per_launch"] = _replay_ms(main, ksteps, 0) / ksteps
+    del main
+    if op.launches > 1:
+        prep = _graph_set(op, xs, ys, ct.PART_PREPARE)
+        for j in range(3):
+            prep[j % nsets].replay()
+        torch.cuda.synchronize(device)
+        info["prepare_ms_per_call"] = _replay_ms(prep, ksteps, 0) / ksteps
+        del prep
+    else:
+        info["prepare_ms_per_call"] = 0.0
+    # leave Y as the full call writes it (the parts runs above overwrote it)
+    for i in range(nsets):
+        op(xs[i], out=ys[i])
+    torch.cuda.synchronize(device)
     return ms, info
+
+
+def kernel_roofline(wl, wid, info, call_seconds, peaks, sms):
+    """The roofline object of a workload: the dominant (main) kernel timed
+    alone against its bound, with the whole call beside it."""
+    flop, nbytes = workload_numbers(wl)
+    ksec = info["kernel_ms_per_launch"] / 1e3
+    roof = roofline_for(wl, ksec, peaks, sms, info["kernel"])
+    roof["peak_source"] = peaks["source"] + " (burst)"
+    roof["kernel_us"] = ksec * 1e6
+    roof["prepare_us"] = info["prepare_ms_per_call"] * 1e3
+    call = roofline_for(wl, call_seconds, peaks, sms, info["kernel"])
+    roof["call"] = {"us": call_seconds * 1e6, "achieved": call["achieved"], "frac": call["frac"],
+                    "tensor_frac": call.get("tensor_frac"), "hbm_frac": call.get("hbm_frac")}
+    roof["algorithmic"] = {"flop": flop, "bytes": nbytes}
+    return annotate_roofline(roof, wid, info["kernel"], info["launches_per_step"], nbytes=nbytes)
 
 
 def make_dist_max(dist, device=None):
@@ -409,13 +473,15 @@ GENERAL_SHAPES = [
 
 
 def general_shapes(device, peaks, runs=50, algos=("auto", "dense_tc", "dense_tc_pertap",
-                                                  "dense_tc_pair", "generic"), only=None):
+                                                  "dense_tc_pair", "generic"), only=None,
+                   quiet=False):
     """Device time per call of each general shape under each algorithm that
     accepts it (CUDA events around a batch of calls, inputs rotated so the
     outputs exceed L2): kernel, effective TFLOP/s and the roofline of the
     binding resource (tensor peak for the dtype, 3xTF32 for fp32, or HBM for
     the algorithmic bytes X + W + bias + Y)."""
     torch.cuda.set_device(device)
+    results = []
     for si, (name, xs, ws, dt, layout, kw) in enumerate(GENERAL_SHAPES):
         if only is not None and si != only:
             continue
@@ -457,11 +523,15 @@ def general_shapes(device, peaks, runs=50, algos=("auto", "dense_tc", "dense_tc_
             t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
             bound = "tensor" if t_tc >= t_hbm else "hbm"
             frac = max(t_tc, t_hbm) / (us * 1e-6)
-            print(json.dumps({"shape": name, "algo": algo, "kernel": op.kernel,
-                              "us_per_call": round(us, 2), "tflops": round(flop / us / 1e6, 1),
-                              "gbs": round(nbytes / us / 1e3, 1), "bound": bound,
-                              "frac": round(frac, 3)}), flush=True)
+            rec = {"shape": name, "algo": algo, "kernel": op.kernel,
+                   "us_per_call": round(us, 2), "tflops": round(flop / us / 1e6, 1),
+                   "gbs": round(nbytes / us / 1e3, 1), "bound": bound,
+                   "frac": round(frac, 3)}
+            results.append(rec)
+            if not quiet:
+                print(json.dumps(rec), flush=True)
             del op, xd, yd
+    return results
 
 
 def main():
@@ -560,10 +630,7 @@ def main():
     ms, info = time_device(wl, device, args.steps, args.warmup, l2, dist_max, sampler)
     ms, value = aggregate(flop, ms, args.steps, world, dist_max)
     sec_per_step = ms / 1e3 / args.steps
-    roof = roofline_for(wl, sec_per_step, peaks, props.multi_processor_count, info["kernel"])
-    roof["peak_source"] = peaks["source"] + " (burst)"
-    annotate_roofline(roof, args.workload, info["kernel"], info["launches_per_step"])
-    roof["per_call_us"] = sec_per_step * 1e6
+    roof = kernel_roofline(wl, args.workload, info, sec_per_step, peaks, props.multi_processor_count)
 
     e2e_steps = max(3, min(args.steps, 50))
     ems, hb, db = time_e2e(wl, device, e2e_steps, 3)
@@ -581,11 +648,13 @@ def main():
             if dist_max is not None:
                 oms = dist_max("max", oms)
             osec = oms / 1e3 / osteps
-            oroof = roofline_for(owl, osec, peaks, props.multi_processor_count, oinfo["kernel"])
-            annotate_roofline(oroof, wid, oinfo["kernel"], oinfo["launches_per_step"])
+            oroof = kernel_roofline(owl, wid, oinfo, osec, peaks, props.multi_processor_count)
             others[str(wid)] = {"workload": owl.name, "kernel": oinfo["kernel"],
                                 "us_per_step": osec * 1e6, "tflops": ofl / osec / 1e12,
                                 "roofline": oroof}
+        if world == 1:
+            others["general"] = general_shapes(device, peaks, runs=50, algos=("auto",),
+                                               quiet=True)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -69,17 +69,36 @@ def test_traffic_record_needs_unchanged_source(tmp_path, monkeypatch):
     src.write_bytes(b"kernel source v1\n")
     h = hashlib.sha256(src.read_bytes()).hexdigest()[:16]
     rec = {"2": {"kernel": "dense_tc_pair", "source": "k_x.cu", "sha256_16": h,
-                 "bytes_per_launch": 123, "share_of_call": 0.8}}
+                 "dram_read": 100, "dram_write": 23, "bytes_per_launch": 123}}
     (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(rec))
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     assert bench.traffic_for(2, "dense_tc_pair") == 123
     assert bench.traffic_for(2, "dense_tc") is None           # another kernel
     assert bench.traffic_for(3, "dense_tc_pair") is None      # another workload
-    roof = bench.annotate_roofline(dict(frac=0.4), 2, "dense_tc_pair", 2)
-    assert roof["kernel_share_of_call"] == 0.8
-    assert roof["kernel_frac_est"] == pytest.approx(0.5)
+    roof = bench.annotate_roofline(dict(frac=0.4), 2, "dense_tc_pair", 2, nbytes=246)
+    assert roof["traffic"] == 123
+    assert roof["traffic_detail"] == {"dram_read": 100, "dram_write": 23}
+    assert roof["traffic_over_algorithmic"] == pytest.approx(0.5)
     src.write_bytes(b"kernel source v2\n")                     # the kernel changed
     assert bench.traffic_for(2, "dense_tc_pair") is None
     roof = bench.annotate_roofline(dict(frac=0.4), 2, "dense_tc_pair", 2)
-    assert roof["traffic"] is None and "kernel_frac_est" not in roof
+    assert roof["traffic"] is None and "traffic_detail" not in roof
 
+
+def test_kernel_roofline_uses_the_kernel_time():
+    """achieved/frac come from the main kernel timed alone; the whole call is
+    reported beside it, with both fractions for the fp16 workloads."""
+    info = dict(kernel="dense_tc_pair", kernel_ms_per_launch=0.030, prepare_ms_per_call=0.008,
+                launches_per_step=2)
+    f2, b2 = bench.workload_numbers(WORKLOADS[2])
+    r = bench.kernel_roofline(WORKLOADS[2], 2, info, 40e-6, PEAKS, 148)
+    assert r["achieved"] == pytest.approx(f2 / 30e-6 / 1e12)
+    assert r["kernel_us"] == pytest.approx(30.0) and r["prepare_us"] == pytest.approx(8.0)
+    assert r["call"]["us"] == pytest.approx(40.0)
+    assert r["call"]["frac"] == pytest.approx(f2 / 40e-6 / 1e12 / 1662.5)
+    assert r["call"]["hbm_frac"] == pytest.approx(b2 / 40e-6 / 1e9 / 6541.8)
+    info3 = dict(info, kernel="dense_tc")
+    f3, b3 = bench.workload_numbers(WORKLOADS[3])
+    r = bench.kernel_roofline(WORKLOADS[3], 3, info3, 40e-6, PEAKS, 148)
+    assert r["bound"] == "hbm"
+    assert r["tensor_frac"] == pytest.approx(f3 / 30e-6 / 1e12 / 1662.5)
