@@ -623,3 +623,31 @@ def test_multi_device_batch_split():
     xa, wa, ba = to_oracle(x, w, b, "nchw")
     ref, absacc = conv_transpose_ref(xa, wa, ba, attrs_from(case))
     check_close(y, ref, absacc, torch.float16, "multi-device batch split")
+
+
+@pytest.mark.parametrize("case", [
+    # the 3-D upsample's attributes: J_x 12 of a 32-wide row segment, ragged y and z
+    dict(x_shape=[2, 64, 6, 7, 12], w_shape=[64, 32, 3, 3, 3], strides=[2, 2, 2],
+         pads=[1, 1, 1, 1, 1, 1], output_padding=[1, 1, 1]),
+    # odd out_y (the last row's second y phase lies outside Y), bias
+    dict(x_shape=[1, 32, 4, 5, 8], w_shape=[32, 16, 3, 3, 3], strides=[2, 2, 2],
+         pads=[1, 1, 1, 1, 1, 1], output_padding=[1, 0, 1], bias=True),
+    # 2-D decoder-like: 64-wide rows (two warps per row), M = 72 (a one-chunk channel block)
+    dict(x_shape=[2, 32, 5, 64], w_shape=[32, 72, 4, 4], strides=[2, 2], pads=[1, 1, 1, 1], bias=True),
+    # J_x = 200: two x tiles of 128 (kernel 2, stride 2: one tap per phase)
+    dict(x_shape=[1, 16, 3, 200], w_shape=[16, 24, 2, 2], strides=[2, 2], bias=True),
+    # stride 1 along x (one x phase per store), M = 40
+    dict(x_shape=[2, 32, 10, 24], w_shape=[32, 40, 3, 3], strides=[1, 1], pads=[1, 1, 1, 1], bias=True),
+    # 1-D, 100 positions per row
+    dict(x_shape=[2, 64, 100], w_shape=[64, 32, 4], strides=[2], pads=[1, 1], bias=True),
+    # 20 positions per row, C = 136 (three channel blocks)
+    dict(x_shape=[2, 136, 9, 20], w_shape=[136, 48, 4, 4], strides=[2, 2], pads=[1, 1, 1, 1], bias=True),
+])
+def test_dense_tc_row_mode(case):
+    """The halo kernel's row mode (whole output rows per unit, one TMA box per
+    x offset, epilogue tiles written by TMA tensor stores with the parts
+    outside Y clipped): channels-first fp16 shapes with every phase live and
+    out_x a multiple of 8, identity and ReLU."""
+    full_parity(case, torch.float16, 97, "nchw", algo="dense_tc", expect_kernel="dense_tc")
+    full_parity(dict(case, activation="relu"), torch.float16, 98, "nchw", algo="dense_tc",
+                expect_kernel="dense_tc")

@@ -26,11 +26,21 @@
 // channels as two 16-byte vectors channels-last).  More epilogue warps were
 // measured slower here: the register cap of a larger block costs the 3-D
 // upsample more than the extra store parallelism gains.
+//
+// Row mode (channels-first output with s_x = 1 or paired x phases, every
+// phase live, out_x a multiple of 8): positions are numbered without halo
+// columns (pitch BXt = 32, 64 or 128), one TMA box per x offset, and a unit
+// is R = Mt*128/BXt whole rows.  Each epilogue warp then owns 32 consecutive
+// J_x of one row: it writes the outputs of one (z phase, y phase, 32-channel
+// block) as a [32 channels][s_x*32 x] tile to shared memory and one lane
+// stores the tile with a TMA tensor store (parts outside Y are clipped), so
+// the output leaves the SM as whole lines from the bulk-copy engine.
 #include <cuda.h>
 
 #include <algorithm>
 #include <array>
 #include <atomic>
+#include <cstring>
 #include <vector>
 
 #include "ct_cuda_util.h"
@@ -43,9 +53,13 @@ namespace {
 constexpr int kMaxPhases = 64;
 constexpr int kMaxGroups = 64;
 constexpr int kMaxItems = 512;
+constexpr int kMaxZ = 8;   // row mode: z slices of one unit's input
 constexpr int kThreads = 256;
 constexpr int kEpiSets = (kThreads / 32 - 4) / 4;   // epilogue warps per TMEM lane quarter
 constexpr int kSmemBudget = 227 * 1024;
+// row mode: per epilogue warp two output tiles of 32 channels x 64 halves
+constexpr int kStageTile = 32 * 64 * 2;
+constexpr int kStageBytes = (kThreads / 32 - 4) * 2 * kStageTile;
 
 struct Item {
     int16_t e[3];       // input offset (z, y, x)
@@ -66,11 +80,17 @@ struct HaloTables {
     int32_t TX, PU, n_units, n_groups;  // x tiles, units per (n, z, x-tile) plane
     int32_t nbuf, bufcols, SA, SB, a_bytes, a_stride, b_slot_bytes, BR;
     int32_t resident, res_rows;
+    int32_t rowmode, n_ex, box_rows, R;  // row mode: x-offset boxes, rows per unit
+    int32_t zslices;                     // A ring entries per channel block (row mode: z slices)
     int32_t nhwc, has_bias, dead, pair_x, act;
     int32_t n_phases, n_items, total_rows;
     int16_t phase_r[kMaxPhases][3];
     int16_t g_phase0[kMaxGroups], g_nphase[kMaxGroups], g_item0[kMaxGroups], g_nitem[kMaxGroups];
     int16_t g_emin[kMaxGroups][3];      // smallest input offset of the group's taps
+    // row mode: the input comes in z slices (zslices per channel block), and
+    // a group's items are ordered by z offset; its items of slice z are
+    // [g_zitem[g][z], g_zitem[g][z + 1]) relative to g_item0
+    int16_t g_zitem[kMaxGroups][kMaxZ + 1];
     int32_t g_brow[kMaxGroups], g_rows_kb[kMaxGroups];
     Item item[kMaxItems];
 };
@@ -136,6 +156,13 @@ struct SItem {
     int32_t shift;
     int32_t brow;
     int16_t n, tcol, first, pad;
+};
+// An item as the MMA loop consumes it: descriptor offsets in 16-byte units
+// (A rows from the tile start, B rows from the channel block's weights), the
+// instruction descriptor, and the accumulator column with the first-write
+// flag in bit 16.
+struct MItem {
+    uint32_t a16, b16, idesc, col_first;
 };
 struct SGroup {
     int32_t brow, rows_kb;
@@ -207,8 +234,8 @@ __device__ __forceinline__ void store_chunk16(__half *dst, long long stride, con
 template <int ACT>
 __global__ void __launch_bounds__(kThreads, 1)
     dense_halo_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                      const __grid_constant__ HaloTables T, const __half *__restrict__ bias,
-                      __half *__restrict__ y) {
+                      const __grid_constant__ CUtensorMap tmY, const __grid_constant__ HaloTables T,
+                      const __half *__restrict__ bias, __half *__restrict__ y) {
     using namespace sm100;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -220,13 +247,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int res_rows = T.res_rows, BXt = T.BXt, HX = T.HX, nhwc = T.nhwc, pair_x = T.pair_x;
     const int n_items = T.n_items, n_groups = T.n_groups, n_phases = T.n_phases;
     const Geo G{T.n_groups, T.PU, T.TX, T.nJ[0], T.Mt, T.HX};
+    const int rowmode = T.rowmode, n_ex = T.n_ex, box_rows = T.box_rows, zslices = T.zslices;
     // shared-memory layout
     uint8_t *sA = smem;
-    uint8_t *sB = sA + (size_t)SA * a_stride;       // ring slots, or the resident weights
+    uint8_t *sStage = sA + (size_t)SA * a_stride;   // row mode: output tiles, two per epilogue warp
+    uint8_t *sB = sStage + (rowmode ? (size_t)kStageBytes : 0);   // ring slots, or the resident weights
     const size_t b_region = resident ? (size_t)res_rows * 128 : (size_t)SB * b_slot;
     float *bias_s = reinterpret_cast<float *>(sB + b_region);
     SItem *items_s = reinterpret_cast<SItem *>(bias_s + ((Np + 31) & ~31));   // bias padded to 32
-    SGroup *groups_s = reinterpret_cast<SGroup *>(items_s + n_items);
+    MItem *mitems_s = reinterpret_cast<MItem *>(items_s + n_items);
+    SGroup *groups_s = reinterpret_cast<SGroup *>(mitems_s + n_items);
     int16_t *phr_s = reinterpret_cast<int16_t *>(groups_s + n_groups);
     uint64_t *bars = reinterpret_cast<uint64_t *>(((uintptr_t)(phr_s + 3 * n_phases) + 7) & ~(uintptr_t)7);
     const uint32_t fullA = smem_u32(bars), emptyA = smem_u32(bars + SA);
@@ -255,6 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_barrier_init();
         prefetch_tmap(&tmA);
         prefetch_tmap(&tmB);
+        if (rowmode) prefetch_tmap(&tmY);
     }
     for (int i = threadIdx.x; i < n_items; i += kThreads) {
         SItem it;
@@ -265,6 +296,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         it.first = T.item[i].first;
         it.pad = 0;
         items_s[i] = it;
+        MItem mi;
+        mi.a16 = (uint32_t)it.shift * 8u;
+        mi.b16 = (uint32_t)it.brow * 8u;
+        mi.idesc = idesc_f16_f32(128, it.n);
+        mi.col_first = (uint32_t)it.tcol | ((uint32_t)(it.first ? 1 : 0) << 16);
+        mitems_s[i] = mi;
     }
     for (int g = threadIdx.x; g < n_groups; g += kThreads) {
         SGroup gr;
@@ -304,14 +341,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int x0 = U.tx * BXt + gr.emin[2];
             const int y0 = U.y0 + gr.emin[1];
             const int z0 = U.jz + gr.emin[0];
-            for (int kb = 0; kb < KB; ++kb, ++ia) {
+            for (int q = 0; q < KB * zslices && ok; ++q, ++ia) {
+                const int kb = q / zslices, z = q - kb * zslices;
                 const int s = ia % SA;
                 if (ia >= SA && !mbar_wait(emptyA + 8 * s, ((ia / SA) - 1) & 1, err, 1)) {
                     ok = false;
                     break;
                 }
                 mbar_arrive_expect_tx(fullA + 8 * s, a_bytes);
-                tma_load_5d(smem_u32(sA + (size_t)s * a_stride), &tmA, fullA + 8 * s, kb * 64, x0, y0, z0, U.n);
+                if (rowmode) {
+                    // one z slice: one box per x offset, the unit's rows at pitch BXt
+                    for (int e = 0; e < n_ex; ++e)
+                        tma_load_5d(smem_u32(sA + (size_t)s * a_stride + (size_t)e * box_rows * 128), &tmA,
+                                    fullA + 8 * s, kb * 64, x0 + e, y0, z0 + z, U.n);
+                } else {
+                    tma_load_5d(smem_u32(sA + (size_t)s * a_stride), &tmA, fullA + 8 * s, kb * 64, x0, y0, z0, U.n);
+                }
             }
         }
         const int first = ia > SA ? ia - SA : 0;
@@ -356,11 +401,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 1) {
         // ---------------- MMA issue ----------------
-        // The whole warp walks the loop, so every descriptor it computes is
-        // warp-uniform (items are read from the kernel parameters with uniform
-        // indices, ring positions advance by counters); one elected lane
-        // issues the MMAs and commits.  A single-lane loop cannot keep narrow
-        // MMAs back to back.
+        // One elected lane walks the items and issues (the rest of the warp
+        // waits at the end of each channel block).  The items are narrow
+        // (down to N = 32, four K steps each): a whole-warp loop, with its
+        // reconvergence between items, measured twice as long per unit here.
+        // Each item's descriptor offsets are precomputed in shared memory;
+        // the lane adds them to the descriptors of the tile and the weights.
         const bool issuer = elect_one();
         bool ok = true;
         if (resident) ok = __all_sync(0xffffffffu, mbar_wait(bres, 0, err, 6));
@@ -378,41 +424,52 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t dbase = tmem_base + buf * bufcols;
             const uint32_t mstep = (uint32_t)(T.g_nphase[U.g] * Np);
             const int rel = U.F0 - U.y0 * HX;   // row of the unit's first position in the tile
-            for (int kb = 0; kb < KB; ++kb) {
-                ok = __all_sync(0xffffffffu, mbar_wait(fullA + 8 * sa_slot, sa_phase, err, 8));
-                if (!ok) break;
-                tc_fence_after();
-                const uint32_t a_addr = smem_u32(sA) + sa_slot * (uint32_t)a_stride + (uint32_t)rel * 128;
-                const uint32_t bres_base = smem_u32(sB) + (uint32_t)((gbrow + kb * grows) * 128);
-                for (int it = i0; it < i1; ++it) {
-                    uint32_t b_addr;
-                    if (resident) {
-                        b_addr = bres_base + (uint32_t)T.item[it].brow * 128;
+            for (int q = 0; q < KB * zslices && ok; ++q) {
+                const int kb = q / zslices, z = q - kb * zslices;
+                // the items that read this ring entry: all of the group's, or
+                // (row mode) those of z slice z
+                const int j0 = rowmode ? i0 + T.g_zitem[U.g][z] : i0;
+                const int j1 = rowmode ? i0 + T.g_zitem[U.g][z + 1] : i1;
+                if (issuer) {
+                    ok = mbar_wait(fullA + 8 * sa_slot, sa_phase, err, 8);
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(sA) + sa_slot * (uint32_t)a_stride + (uint32_t)rel * 128;
+                    const uint64_t adesc0 = desc_kmajor_sw128(a_addr);
+                    const uint64_t bdesc0 = desc_kmajor_sw128(smem_u32(sB) + (uint32_t)((gbrow + kb * grows) * 128));
+                    if (resident && ok) {
+                        // weights resident: nothing to wait for between the items
+                        for (int it = j0; it < j1; ++it) {
+                            const MItem mi = mitems_s[it];
+                            const uint64_t ad = adesc0 + mi.a16;
+                            const uint64_t bd = bdesc0 + mi.b16;
+                            const uint32_t d = dbase + (mi.col_first & 0xffffu);
+                            const uint32_t acc0 = (kb == 0 && (mi.col_first >> 16)) ? 0u : 1u;
+                            issue4(d, ad, bd, mi.idesc, acc0);
+                            if (Mt > 1) issue4(d + mstep, ad + 1024, bd, mi.idesc, acc0);   // +128 rows
+                        }
                     } else {
-                        ok = __all_sync(0xffffffffu, mbar_wait(fullB + 8 * sb_slot, sb_phase, err, 9));
-                        if (!ok) break;
-                        tc_fence_after();
-                        b_addr = smem_u32(sB) + sb_slot * (uint32_t)b_slot;
+                        for (int it = j0; it < j1 && ok; ++it) {
+                            const MItem mi = mitems_s[it];
+                            ok = mbar_wait(fullB + 8 * sb_slot, sb_phase, err, 9);
+                            if (!ok) break;
+                            tc_fence_after();
+                            const uint64_t bd = desc_kmajor_sw128(smem_u32(sB) + sb_slot * (uint32_t)b_slot);
+                            const uint64_t ad = adesc0 + mi.a16;
+                            const uint32_t d = dbase + (mi.col_first & 0xffffu);
+                            const uint32_t acc0 = (kb == 0 && (mi.col_first >> 16)) ? 0u : 1u;
+                            issue4(d, ad, bd, mi.idesc, acc0);
+                            if (Mt > 1) issue4(d + mstep, ad + 1024, bd, mi.idesc, acc0);   // +128 rows
+                            mma_commit(emptyB + 8 * sb_slot);
+                            if (++sb_slot == (uint32_t)SB) {
+                                sb_slot = 0;
+                                sb_phase ^= 1u;
+                            }
+                        }
                     }
-                    const uint64_t bd = desc_kmajor_sw128(b_addr);
-                    const uint64_t ad = desc_kmajor_sw128(a_addr + (uint32_t)T.item[it].shift * 128);
-                    const uint32_t idesc = idesc_f16_f32(128, T.item[it].n);
-                    const uint32_t d = dbase + (uint32_t)T.item[it].tcol;
-                    const uint32_t acc0 = (kb == 0 && T.item[it].first) ? 0u : 1u;
-                    if (issuer) {
-                        issue4(d, ad, bd, idesc, acc0);
-                        if (Mt > 1) issue4(d + mstep, ad + 1024, bd, idesc, acc0);   // +128 rows
-                        if (!resident) mma_commit(emptyB + 8 * sb_slot);
-                    }
-                    __syncwarp();
-                    if (!resident && ++sb_slot == (uint32_t)SB) {
-                        sb_slot = 0;
-                        sb_phase ^= 1u;
-                    }
+                    if (ok) mma_commit(emptyA + 8 * sa_slot);
                 }
-                if (!ok) break;
-                if (issuer) mma_commit(emptyA + 8 * sa_slot);
                 __syncwarp();
+                ok = __all_sync(0xffffffffu, ok);
                 if (++sa_slot == (uint32_t)SA) {
                     sa_slot = 0;
                     sa_phase ^= 1u;
@@ -425,6 +482,117 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (issuer) mma_commit(mdone);
         __syncwarp();
         mbar_wait(mdone, 0, err, 10);
+    } else if (warp >= 4 && rowmode) {
+        // ---------------- epilogue, row mode: tiles to shared memory, TMA stores ----------------
+        const int q = warp & 3;                  // the TMEM lane quarter this warp may read
+        const int sx = T.s[2];
+        const bool has_bias = T.has_bias;
+        const bool bias_vec = has_bias && (reinterpret_cast<uintptr_t>(bias) & 15) == 0;
+        uint8_t *stage = sStage + (size_t)(warp - 4) * 2 * kStageTile;
+        int sbuf = 0;
+        int local = 0;
+        for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++local) {
+            const Unit U = decode_unit(G, u);
+            const int buf = nbuf == 2 ? (local & 1) : 0;
+            const int use = nbuf == 2 ? (local >> 1) : local;
+            if (!mbar_wait(tfull + 8 * buf, use & 1, err, 12)) break;
+            tc_fence_after();
+            const uint32_t dbase = tmem_base + ((uint32_t)(32 * q) << 16) + buf * bufcols;
+            const int gcols = T.g_nphase[U.g] * Np;
+            const int ph0 = T.g_phase0[U.g], ph1 = ph0 + T.g_nphase[U.g];
+            for (int mt = 0; mt < Mt; ++mt) {
+                const int p0 = mt * 128 + 32 * q;          // this warp's first position in the unit
+                const int jy = U.y0 + p0 / BXt;
+                const int jx0 = U.tx * BXt + p0 % BXt;
+                for (int ph = ph0; ph < ph1; ph += sx) {   // s_x = 2: (ph, ph + 1) have r_x = 0, 1
+                    const int oz = T.s[0] * U.jz + T.phase_r[ph][0];
+                    const int oy = T.s[1] * jy + T.phase_r[ph][1];
+                    const uint32_t col0 = dbase + mt * gcols + (ph - ph0) * Np;
+                    for (int m0 = 0; m0 < Np; m0 += 32) {
+                        uint32_t v0[16], v1[16], w0[16], w1[16];
+                        const bool two = m0 + 16 < Np;
+                        tmem_ld16(col0 + m0, v0);
+                        if (two) tmem_ld16(col0 + m0 + 16, v1);
+                        if (sx == 2) {
+                            tmem_ld16(col0 + Np + m0, w0);
+                            if (two) tmem_ld16(col0 + Np + m0 + 16, w1);
+                        }
+                        tmem_ld_wait();
+                        // the bias from global memory (read-only path): shared-memory
+                        // reads here would queue behind the tile loads and stores
+                        float bb[32];
+                        if (bias_vec && m0 + 32 <= M) {
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                const uint4 h = __ldg(reinterpret_cast<const uint4 *>(bias + m0) + j);
+                                const __half2 *h2 = reinterpret_cast<const __half2 *>(&h);
+#pragma unroll
+                                for (int c = 0; c < 4; ++c) {
+                                    const float2 f = __half22float2(h2[c]);
+                                    bb[8 * j + 2 * c] = f.x;
+                                    bb[8 * j + 2 * c + 1] = f.y;
+                                }
+                            }
+                        } else if (!has_bias) {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) bb[j] = 0.f;
+                        } else {   // the last, partial block of channels, or an unaligned bias
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) bb[j] = m0 + j < M ? __half2float(__ldg(bias + m0 + j)) : 0.f;
+                        }
+                        // the tile written two stores ago must have been read out
+                        if (lane == 0) bulk_wait_group_read<1>();
+                        __syncwarp();
+                        uint8_t *tile = stage + (size_t)sbuf * kStageTile;
+                        if (sx == 2) {
+                            // [32 channels][64 x]: lane = J_x, its two x phases side by side
+                            uint32_t *t32 = reinterpret_cast<uint32_t *>(tile) + lane;
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) {
+                                const __half2 h = __floats2half2_rn(apply_act(__uint_as_float(v0[j]) + bb[j], ACT),
+                                                                    apply_act(__uint_as_float(w0[j]) + bb[j], ACT));
+                                t32[32 * j] = *reinterpret_cast<const uint32_t *>(&h);
+                            }
+                            if (two) {
+#pragma unroll
+                                for (int j = 0; j < 16; ++j) {
+                                    const __half2 h =
+                                        __floats2half2_rn(apply_act(__uint_as_float(v1[j]) + bb[16 + j], ACT),
+                                                          apply_act(__uint_as_float(w1[j]) + bb[16 + j], ACT));
+                                    t32[32 * (16 + j)] = *reinterpret_cast<const uint32_t *>(&h);
+                                }
+                            }
+                        } else {
+                            // [32 channels][32 x]
+                            __half *t16 = reinterpret_cast<__half *>(tile) + lane;
+#pragma unroll
+                            for (int j = 0; j < 16; ++j)
+                                t16[32 * j] = __float2half_rn(apply_act(__uint_as_float(v0[j]) + bb[j], ACT));
+                            if (two) {
+#pragma unroll
+                                for (int j = 0; j < 16; ++j)
+                                    t16[32 * (16 + j)] =
+                                        __float2half_rn(apply_act(__uint_as_float(v1[j]) + bb[16 + j], ACT));
+                            }
+                        }
+                        fence_proxy_async();   // the tile, written by this warp, before the bulk store reads it
+                        __syncwarp();
+                        if (lane == 0) {
+                            // channels m0 + 16.. of a one-chunk piece hold no data: they lie at or
+                            // beyond M, where the store writes nothing
+                            tma_store_5d(&tmY, smem_u32(tile), sx * jx0, oy, oz, m0, U.n);
+                            bulk_commit_group();
+                        }
+                        sbuf ^= 1;
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty + 8 * buf);
+        }
+        if (lane == 0) bulk_wait_group_all();   // every store has left this CTA's shared memory
+        __syncwarp();
     } else if (warp >= 4) {
         // ---------------- epilogue ----------------
         const int lane_base = 32 * (warp & 3);   // the TMEM lane quarter this warp may read
@@ -555,16 +723,29 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 size_t smem_bytes(const HaloTables &T) {
     const size_t b_region = T.resident ? (size_t)T.res_rows * 128 : (size_t)T.SB * T.b_slot_bytes;
-    const size_t tables = (size_t)T.n_items * sizeof(SItem) + (size_t)T.n_groups * sizeof(SGroup) +
+    const size_t tables = (size_t)T.n_items * (sizeof(SItem) + sizeof(MItem)) + (size_t)T.n_groups * sizeof(SGroup) +
                           (size_t)T.n_phases * 6 + 8;
-    return 1024 + (size_t)T.SA * T.a_stride + b_region + (size_t)((T.Np + 31) & ~31) * 4 + tables +
-           (size_t)(2 * T.SA + 2 * T.SB + 6) * 8 + 16;
+    return 1024 + (size_t)T.SA * T.a_stride + (T.rowmode ? (size_t)kStageBytes : 0) + b_region +
+           (size_t)((T.Np + 31) & ~31) * 4 + tables + (size_t)(2 * T.SA + 2 * T.SB + 6) * 8 + 16;
+}
+
+// Row mode applies to channels-first output whose x phases the epilogue can
+// store as contiguous runs: s_x = 1, or s_x = 2 with both x phases live;
+// every phase live (the stores cover whole rows); out_x a multiple of 8 (the
+// output rows are 16-byte multiples, as TMA needs).
+bool rowmode_ok(const Plan &p) {
+    if (p.layout != CT_NCHW || has_dead_phases(p)) return false;
+    if (!(p.s[2] == 1 || (p.s[2] == 2 && p.out[2] % 2 == 0))) return false;
+    if (p.out[2] % 8 != 0) return false;
+    for (int a = 0; a < 3; ++a)
+        if (p.out[a] > (1 << 30) / 2) return false;
+    return true;
 }
 
 // Build the tables for one policy: Mt M-tiles per unit and groups of at
 // most `gmax_cols` accumulator columns.  Returns false when a limit or the
 // shared-memory budget is exceeded.
-bool build_tables(const Plan &p, HaloTables &T, int Mt, int gmax_cols) {
+bool build_tables(const Plan &p, HaloTables &T, int Mt, int gmax_cols, bool rowmode) {
     T.N = (int32_t)p.N;
     T.C = (int32_t)p.C;
     T.M = (int32_t)p.M;
@@ -575,6 +756,9 @@ bool build_tables(const Plan &p, HaloTables &T, int Mt, int gmax_cols) {
     T.act = p.act;
     T.Mt = Mt;
     if (T.Np > gmax_cols) return false;
+    // row mode stores the x phases of a (z, y) phase pair together: both must
+    // fall in one group
+    if (rowmode && p.s[2] * T.Np > gmax_cols) return false;
     for (int a = 0; a < 3; ++a) {
         T.out[a] = (int32_t)p.out[a];
         T.s[a] = (int32_t)p.s[a];
@@ -645,17 +829,39 @@ bool build_tables(const Plan &p, HaloTables &T, int Mt, int gmax_cols) {
         }
     }
     // input tile geometry
-    if (T.nJ[2] + T.span[2] <= 256) {
-        T.BXt = T.nJ[2];
+    T.rowmode = rowmode ? 1 : 0;
+    if (rowmode) {
+        // pitch BXt (no halo columns): 32, 64 or 128 J_x per row segment, x
+        // tiles of 128 beyond that; R whole rows per unit
+        T.BXt = T.nJ[2] <= 32 ? 32 : T.nJ[2] <= 64 ? 64 : 128;
+        T.HX = T.BXt;
+        T.R = Mt * 128 / T.BXt;
+        T.HYb = T.R + T.span[1];
+        T.n_ex = 1 + T.span[2];
     } else {
-        T.BXt = 256 - T.span[2];
-        if (T.BXt < 64) return false;
+        if (T.nJ[2] + T.span[2] <= 256) {
+            T.BXt = T.nJ[2];
+        } else {
+            T.BXt = 256 - T.span[2];
+            if (T.BXt < 64) return false;
+        }
+        T.HX = T.BXt + T.span[2];
+        T.HYb = (int32_t)ceil_div((int64_t)Mt * 128 + T.HX + T.span[2], T.HX) + T.span[1];
+        T.R = 0;
+        T.n_ex = 1;
     }
-    T.HX = T.BXt + T.span[2];
-    T.HYb = (int32_t)ceil_div((int64_t)Mt * 128 + T.HX + T.span[2], T.HX) + T.span[1];
     T.HZb = 1 + T.span[0];
     if (T.HYb > 256 || T.HZb > 256) return false;
-    T.a_bytes = T.HX * T.HYb * T.HZb * 128;
+    if (rowmode) {
+        // one ring entry per z slice: n_ex boxes of HX x HYb positions
+        if (T.HZb > kMaxZ) return false;
+        T.zslices = T.HZb;
+        T.box_rows = T.HX * T.HYb;
+    } else {
+        T.zslices = 1;
+        T.box_rows = T.HX * T.HYb * T.HZb;
+    }
+    T.a_bytes = T.n_ex * T.box_rows * 128;
     T.a_stride = (T.a_bytes + 1023) & ~1023;
     T.TX = (int32_t)ceil_div(T.nJ[2], T.BXt);
     const long long plane_pos = (long long)T.nJ[1] * T.HX;
@@ -665,7 +871,8 @@ bool build_tables(const Plan &p, HaloTables &T, int Mt, int gmax_cols) {
     T.n_units = (int32_t)units;
     // items per group: pairs grouped by input offset, merged over adjacent phases
     int ni = 0, rows_total = 0;
-    const int row_pitch = T.HX, slice_pitch = T.HX * T.HYb;
+    // row mode: a slice holds one z offset (slice_pitch unused), x offsets are boxes
+    const int row_pitch = T.HX, slice_pitch = rowmode ? 0 : T.HX * T.HYb, ex_pitch = rowmode ? T.box_rows : 1;
     for (int g = 0; g < ng; ++g) {
         struct PairRec { int ph, e0, e1, e2; };
         std::vector<PairRec> pairs;
@@ -688,6 +895,9 @@ bool build_tables(const Plan &p, HaloTables &T, int Mt, int gmax_cols) {
         };
         std::stable_sort(offs.begin(), offs.end(),
                          [&](const std::array<int, 3> &a, const std::array<int, 3> &b) { return nph(a) > nph(b); });
+        if (rowmode)   // row mode consumes the input z slice by z slice
+            std::stable_sort(offs.begin(), offs.end(),
+                             [&](const std::array<int, 3> &a, const std::array<int, 3> &b) { return a[0] < b[0]; });
         std::vector<char> touched(np, 0);
         T.g_item0[g] = (int16_t)ni;
         int brow = 0;
@@ -709,7 +919,7 @@ bool build_tables(const Plan &p, HaloTables &T, int Mt, int gmax_cols) {
                 I.e[2] = (int16_t)e[2];
                 I.n = (int16_t)((j - i) * T.Np);
                 I.shift = (e[0] - T.g_emin[g][0]) * slice_pitch + (e[1] - T.g_emin[g][1]) * row_pitch +
-                          (e[2] - T.g_emin[g][2]);
+                          (e[2] - T.g_emin[g][2]) * ex_pitch;
                 I.tcol = (int16_t)((phs[i] - T.g_phase0[g]) * T.Np);
                 I.phase0 = (int16_t)phs[i];
                 I.first = touched[phs[i]] ? 0 : 1;
@@ -722,6 +932,13 @@ bool build_tables(const Plan &p, HaloTables &T, int Mt, int gmax_cols) {
             }
         }
         T.g_nitem[g] = (int16_t)(ni - T.g_item0[g]);
+        if (rowmode) {
+            for (int z = 0; z <= T.zslices; ++z) {
+                int c = 0;
+                while (c < T.g_nitem[g] && T.item[T.g_item0[g] + c].e[0] - T.g_emin[g][0] < z) ++c;
+                T.g_zitem[g][z] = (int16_t)c;
+            }
+        }
         T.g_brow[g] = rows_total;
         T.g_rows_kb[g] = brow;
         rows_total += brow * T.KB;
@@ -742,11 +959,14 @@ bool build_tables(const Plan &p, HaloTables &T, int Mt, int gmax_cols) {
     for (int i = 0; i < ni; ++i) nmax = std::max(nmax, (int)T.item[i].n);
     T.b_slot_bytes = nmax * 128;
     // shared memory: resident weights if they fit next to two input slots
-    const int fixed = 1024 + ((T.Np + 31) & ~31) * 4 + 64 * 8 + 64 + ni * (int)sizeof(SItem) + ng * (int)sizeof(SGroup) +
-                      np * 6 + 8;
+    const int fixed = 1024 + ((T.Np + 31) & ~31) * 4 + 64 * 8 + 64 + ni * (int)(sizeof(SItem) + sizeof(MItem)) + ng * (int)sizeof(SGroup) +
+                      np * 6 + 8 + (rowmode ? kStageBytes : 0);
     T.resident = 0;
     T.res_rows = 0;
-    if ((long long)rows_total * 128 + 2LL * T.a_stride + fixed <= kSmemBudget) {
+    // row mode keeps the weights resident with a single input slot too: its
+    // input is re-read from L2 and the output stores run under the next unit
+    const long long min_sa = rowmode ? 1 : 2;
+    if ((long long)rows_total * 128 + min_sa * T.a_stride + fixed <= kSmemBudget) {
         T.resident = 1;
         T.res_rows = rows_total;
         T.SA = (int)std::min<long long>(4, (kSmemBudget - fixed - (long long)rows_total * 128) / T.a_stride);
@@ -774,10 +994,18 @@ bool build_tables(const Plan &p, HaloTables &T, int Mt, int gmax_cols) {
 // stores, half the weight traffic per pixel) is fastest, then one M-tile with
 // paired phases (double-buffered), then two M-tiles of lone phases.
 bool choose_tables(const Plan &p, HaloTables &T) {
+    if (rowmode_ok(p)) {
+        // row mode: one M-tile per unit, so the accumulators are double-buffered
+        const int ropts[2][2] = {{1, 256}, {1, 128}};
+        for (int o = 0; o < 2; ++o) {
+            T = HaloTables();
+            if (build_tables(p, T, ropts[o][0], ropts[o][1], true)) return true;
+        }
+    }
     const int opts[3][2] = {{2, 256}, {1, 256}, {2, 128}};
     for (int o = 0; o < 3; ++o) {
         T = HaloTables();
-        if (build_tables(p, T, opts[o][0], opts[o][1])) return true;
+        if (build_tables(p, T, opts[o][0], opts[o][1], false)) return true;
     }
     return false;
 }
@@ -843,7 +1071,8 @@ ct_status dense_tc_run(const Plan &p, const void *x, const void *wp, const void 
         const cuuint64_t c2 = (cuuint64_t)p.C * 2;
         const cuuint64_t strides[4] = {c2, c2 * p.in[2], c2 * p.in[2] * p.in[1],
                                        c2 * p.in[2] * p.in[1] * p.in[0]};
-        const cuuint32_t box[5] = {64, (cuuint32_t)T.HX, (cuuint32_t)T.HYb, (cuuint32_t)T.HZb, 1};
+        // row mode loads one z slice per box
+        const cuuint32_t box[5] = {64, (cuuint32_t)T.HX, (cuuint32_t)T.HYb, (cuuint32_t)(T.rowmode ? 1 : T.HZb), 1};
         const cuuint32_t es[5] = {1, 1, 1, 1, 1};
         if (enc(&tmA, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 5, const_cast<void *>(xa), dims, strides, box, es,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -857,6 +1086,23 @@ ct_status dense_tc_run(const Plan &p, const void *x, const void *wp, const void 
         const cuuint32_t es[2] = {1, 1};
         if (enc(&tmB, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(wp), dims, strides, box, es,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return CT_ERR_DEVICE;
+    }
+    CUtensorMap tmY;
+    memset(&tmY, 0, sizeof(tmY));
+    if (T.rowmode) {
+        // Y[n][m][z][y][x] as a 5-D tensor; box: one row segment of s_x*32
+        // outputs for 32 channels
+        const cuuint64_t dims[5] = {(cuuint64_t)p.out[2], (cuuint64_t)p.out[1], (cuuint64_t)p.out[0],
+                                    (cuuint64_t)p.M, (cuuint64_t)p.N};
+        const cuuint64_t e2 = 2;
+        const cuuint64_t strides[4] = {e2 * p.out[2], e2 * p.out[2] * p.out[1], e2 * p.out[2] * p.out[1] * p.out[0],
+                                       e2 * p.out[2] * p.out[1] * p.out[0] * p.M};
+        const cuuint32_t box[5] = {(cuuint32_t)(T.s[2] * 32), 1, 1, 32, 1};
+        const cuuint32_t es[5] = {1, 1, 1, 1, 1};
+        if (enc(&tmY, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 5, y, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return CT_ERR_DEVICE;
     }
@@ -885,11 +1131,11 @@ ct_status dense_tc_run(const Plan &p, const void *x, const void *wp, const void 
     if (T.act == CT_ACT_RELU) {
         static std::atomic<int> attr_set[64];
         if (!allow_smem(dense_halo_kernel<CT_ACT_RELU>, attr_set, kSmemBudget)) return CT_ERR_DEVICE;
-        e = cudaLaunchKernelEx(&cfg, dense_halo_kernel<CT_ACT_RELU>, tmA, tmB, T, b, yy);
+        e = cudaLaunchKernelEx(&cfg, dense_halo_kernel<CT_ACT_RELU>, tmA, tmB, tmY, T, b, yy);
     } else {
         static std::atomic<int> attr_set[64];
         if (!allow_smem(dense_halo_kernel<CT_ACT_IDENTITY>, attr_set, kSmemBudget)) return CT_ERR_DEVICE;
-        e = cudaLaunchKernelEx(&cfg, dense_halo_kernel<CT_ACT_IDENTITY>, tmA, tmB, T, b, yy);
+        e = cudaLaunchKernelEx(&cfg, dense_halo_kernel<CT_ACT_IDENTITY>, tmA, tmB, tmY, T, b, yy);
     }
     if (e != cudaSuccess) {
         cudaGetLastError();

@@ -172,30 +172,37 @@ struct PadGeo {
     int halo_blocks;     // blocks x = 0..halo_blocks-1 write the zero halo
 };
 
-// Halo positions of one image: whole slices outside the input, and in
-// between the rows above and below it and the columns left and right of it.
-struct HaloCount {
-    int top, mid_end, left, right0, lr, n_top, n_mid, h2, ztop, zmid_end;
-    long long n_zt, n_zm, n_all;
-};
+// Zero the halo of one image's padded copy, a padded row (zp, yp) at a time:
+// rows outside the input are zero for their whole width, the others only in
+// the columns left and right of the input.  Warp `wid` of `nw` takes rows
+// round-robin; `zero(pos, q)` writes 16-byte chunk q of padded position pos,
+// `chunks` of them per position.  One row decode per warp and row, then
+// contiguous chunk runs (no per-chunk division beyond the chunk count).
+template <typename F>
+__device__ __forceinline__ void zero_halo_rows(const PadGeo &g, int wid, int nw, int lane, int chunks, F zero) {
+    const int rows = g.HZ * g.HY;
+    const int xl = min(max(g.ox, 0), g.HX);              // left halo columns [0, xl)
+    const int xr = min(max(g.ox + g.W, xl), g.HX);       // right halo columns [xr, HX)
+    for (int row = wid; row < rows; row += nw) {
+        const int zp = row / g.HY, yp = row - zp * g.HY;
+        const bool full = zp < g.oz || zp >= g.oz + g.D || yp < g.oy || yp >= g.oy + g.H;
+        const long long rowpos = (long long)row * g.HX;
+        for (int seg = 0; seg < 2; ++seg) {
+            const int a = full ? (seg == 0 ? 0 : g.HX) : (seg == 0 ? 0 : xr);
+            const int b = full ? (seg == 0 ? g.HX : g.HX) : (seg == 0 ? xl : g.HX);
+            const int nq = (b - a) * chunks;
+            for (int q = lane; q < nq; q += 32) {
+                const int pc = q / chunks;
+                zero(rowpos + a + pc, q - pc * chunks);
+            }
+        }
+    }
+}
 
-__host__ __device__ inline HaloCount halo_count(const PadGeo &g) {
-    HaloCount h;
-    h.top = min(max(g.oy, 0), g.HY);
-    h.mid_end = min(max(g.oy + g.H, h.top), g.HY);
-    h.left = min(max(g.ox, 0), g.HX);
-    h.right0 = min(max(g.ox + g.W, h.left), g.HX);
-    h.lr = h.left + (g.HX - h.right0);
-    h.n_top = h.top * g.HX;
-    h.n_mid = (h.mid_end - h.top) * h.lr;
-    h.h2 = h.n_top + h.n_mid + (g.HY - h.mid_end) * g.HX;
-    h.ztop = min(max(g.oz, 0), g.HZ);
-    h.zmid_end = min(max(g.oz + g.D, h.ztop), g.HZ);
-    const long long P2 = (long long)g.HY * g.HX;
-    h.n_zt = (long long)h.ztop * P2;
-    h.n_zm = (long long)(h.zmid_end - h.ztop) * h.h2;
-    h.n_all = h.n_zt + h.n_zm + (long long)(g.HZ - h.zmid_end) * P2;
-    return h;
+// Blocks that zero the halo: about one warp per padded row.
+inline int halo_blocks_for(const PadGeo &g) {
+    const long long rows = (long long)g.HZ * g.HY;
+    return (int)std::max<long long>(1, std::min<long long>(256, ceil_div(rows, 8)));
 }
 
 __global__ void __launch_bounds__(256) nchw_to_padded_kernel(const __half *__restrict__ x,
@@ -209,39 +216,14 @@ __global__ void __launch_bounds__(256) nchw_to_padded_kernel(const __half *__res
     const int t = threadIdx.x;
     sm100::griddep_launch_dependents();   // the pair kernel may set up while this one runs
     if ((int)blockIdx.x < g.halo_blocks) {
-        // zero halo of image n, channels [c0, c0 + 64), spread over the halo blocks
+        // zero halo of image n, channels [c0, c0 + 64)
         const int c0 = blockIdx.y * kPadC;
         const int c8 = (min(kPadC, Cd - c0)) >> 3;
-        const HaloCount h = halo_count(g);
         __half *img = xp + (long long)n * P * Cd + c0;
-        const long long work = h.n_all * c8;
-        for (long long q = (long long)blockIdx.x * blockDim.x + t; q < work; q += (long long)g.halo_blocks * blockDim.x) {
-            const long long k = q / c8;
-            const int cc = (int)(q - k * c8);
-            long long pos;
-            if (k < h.n_zt || k >= h.n_zt + h.n_zm) {
-                pos = k < h.n_zt ? k : (long long)h.zmid_end * P2 + (k - h.n_zt - h.n_zm);   // whole slice
-            } else {
-                const int kk = (int)(k - h.n_zt);
-                const int zq = kk / h.h2;
-                const int k2 = kk - zq * h.h2;
-                int yp, xq;
-                if (k2 < h.n_top) {
-                    yp = k2 / HX;
-                    xq = k2 - yp * HX;
-                } else if (k2 < h.n_top + h.n_mid) {
-                    const int r = (k2 - h.n_top) / h.lr, j = (k2 - h.n_top) - r * h.lr;
-                    yp = h.top + r;
-                    xq = j < h.left ? j : h.right0 + (j - h.left);
-                } else {
-                    const int k3 = k2 - h.n_top - h.n_mid;
-                    yp = h.mid_end + k3 / HX;
-                    xq = k3 - (k3 / HX) * HX;
-                }
-                pos = (long long)(h.ztop + zq) * P2 + (long long)yp * HX + xq;
-            }
-            *reinterpret_cast<uint4 *>(img + pos * Cd + cc * 8) = make_uint4(0, 0, 0, 0);
-        }
+        zero_halo_rows(g, (int)blockIdx.x * 8 + (t >> 5), g.halo_blocks * 8, t & 31, c8,
+                       [&](long long pos, int q) {
+                           *reinterpret_cast<uint4 *>(img + pos * Cd + q * 8) = make_uint4(0, 0, 0, 0);
+                       });
         return;
     }
     __shared__ __align__(16) __half tile[kPadC][kPadS];
@@ -275,14 +257,25 @@ __global__ void __launch_bounds__(256) nchw_to_padded_kernel(const __half *__res
     {
         const int sl = t >> 3, cv = t & 7;
         const int c = c0 + cv * 8;
+        // this thread's positions are s0 + sl + 32 r: decode the first, then step
+        int iz = (int)(s0 + sl) / (int)HW;                        // S < 2^31
+        int iy = ((int)(s0 + sl) - iz * (int)HW) / W;
+        int ix = (int)(s0 + sl) - iz * (int)HW - iy * W;
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
+            if (r > 0) {
+                ix += 32;
+                while (ix >= W) {
+                    ix -= W;
+                    if (++iy == H) {
+                        iy = 0;
+                        ++iz;
+                    }
+                }
+            }
             const int sp = sl + 32 * r;
             const long long s = s0 + sp;
             if (s >= S || c >= Cd) continue;   // channels C..Cd of the row are zeros
-            const int iz = (int)s / (int)HW;                      // S < 2^31
-            const int rem = (int)s - iz * (int)HW;
-            const int iy = rem / W, ix = rem - iy * W;
             const int zp = iz + g.oz, yp = iy + g.oy, xq = ix + g.ox;
             if (zp < 0 || zp >= g.HZ || yp < 0 || yp >= HY || xq < 0 || xq >= HX) continue;
             __align__(16) __half v[8];
@@ -315,37 +308,13 @@ __global__ void __launch_bounds__(256) nchw_to_padded_f32_kernel(const float *__
     if ((int)blockIdx.x < g.halo_blocks) {
         const int c0 = blockIdx.y * kPadC32;
         const int c4 = (min(kPadC32, Cd - c0)) >> 2;
-        const HaloCount h = halo_count(g);
-        const long long work = h.n_all * c4;
-        for (long long q = (long long)blockIdx.x * blockDim.x + t; q < work; q += (long long)g.halo_blocks * blockDim.x) {
-            const long long k = q / c4;
-            const int cc = (int)(q - k * c4);
-            long long pos;
-            if (k < h.n_zt || k >= h.n_zt + h.n_zm) {
-                pos = k < h.n_zt ? k : (long long)h.zmid_end * P2 + (k - h.n_zt - h.n_zm);
-            } else {
-                const int kk = (int)(k - h.n_zt);
-                const int zq = kk / h.h2;
-                const int k2 = kk - zq * h.h2;
-                int yp, xq;
-                if (k2 < h.n_top) {
-                    yp = k2 / HX;
-                    xq = k2 - yp * HX;
-                } else if (k2 < h.n_top + h.n_mid) {
-                    const int r = (k2 - h.n_top) / h.lr, j = (k2 - h.n_top) - r * h.lr;
-                    yp = h.top + r;
-                    xq = j < h.left ? j : h.right0 + (j - h.left);
-                } else {
-                    const int k3 = k2 - h.n_top - h.n_mid;
-                    yp = h.mid_end + k3 / HX;
-                    xq = k3 - (k3 / HX) * HX;
-                }
-                pos = (long long)(h.ztop + zq) * P2 + (long long)yp * HX + xq;
-            }
-            const long long off = ((long long)n * P + pos) * Cd + c0 + cc * 4;
-            *reinterpret_cast<float4 *>(xh + off) = make_float4(0.f, 0.f, 0.f, 0.f);
-            *reinterpret_cast<float4 *>(xl + off) = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
+        const long long base = (long long)n * P * Cd + c0;
+        zero_halo_rows(g, (int)blockIdx.x * 8 + (t >> 5), g.halo_blocks * 8, t & 31, c4,
+                       [&](long long pos, int q) {
+                           const long long off = base + pos * Cd + q * 4;
+                           *reinterpret_cast<float4 *>(xh + off) = make_float4(0.f, 0.f, 0.f, 0.f);
+                           *reinterpret_cast<float4 *>(xl + off) = make_float4(0.f, 0.f, 0.f, 0.f);
+                       });
         return;
     }
     __shared__ float tile[kPadC32][kPadS + 1];
@@ -416,37 +385,13 @@ __global__ void __launch_bounds__(256) nhwc_to_padded_kernel(const E *__restrict
     const int cch = C / kPer;   // pieces per position
     sm100::griddep_launch_dependents();   // the pair kernel may set up while this one runs
     if ((int)blockIdx.x < g.halo_blocks) {
-        const HaloCount h = halo_count(g);
-        const long long work = h.n_all * cch;
-        for (long long q = (long long)blockIdx.x * blockDim.x + t; q < work; q += (long long)g.halo_blocks * blockDim.x) {
-            const long long k = q / cch;
-            const int cc = (int)(q - k * cch);
-            long long pos;
-            if (k < h.n_zt || k >= h.n_zt + h.n_zm) {
-                pos = k < h.n_zt ? k : (long long)h.zmid_end * P2 + (k - h.n_zt - h.n_zm);
-            } else {
-                const int kk = (int)(k - h.n_zt);
-                const int zq = kk / h.h2;
-                const int k2 = kk - zq * h.h2;
-                int yp, xq;
-                if (k2 < h.n_top) {
-                    yp = k2 / HX;
-                    xq = k2 - yp * HX;
-                } else if (k2 < h.n_top + h.n_mid) {
-                    const int r = (k2 - h.n_top) / h.lr, j = (k2 - h.n_top) - r * h.lr;
-                    yp = h.top + r;
-                    xq = j < h.left ? j : h.right0 + (j - h.left);
-                } else {
-                    const int k3 = k2 - h.n_top - h.n_mid;
-                    yp = h.mid_end + k3 / HX;
-                    xq = k3 - (k3 / HX) * HX;
-                }
-                pos = (long long)(h.ztop + zq) * P2 + (long long)yp * HX + xq;
-            }
-            const long long off = ((long long)n * P + pos) * C + (long long)cc * kPer;
-            *reinterpret_cast<uint4 *>(xh + off) = make_uint4(0, 0, 0, 0);
-            if (xl) *reinterpret_cast<uint4 *>(xl + off) = make_uint4(0, 0, 0, 0);
-        }
+        const long long base = (long long)n * P * C;
+        zero_halo_rows(g, (int)blockIdx.x * 8 + (t >> 5), g.halo_blocks * 8, t & 31, cch,
+                       [&](long long pos, int q) {
+                           const long long off = base + pos * C + (long long)q * kPer;
+                           *reinterpret_cast<uint4 *>(xh + off) = make_uint4(0, 0, 0, 0);
+                           if (xl) *reinterpret_cast<uint4 *>(xl + off) = make_uint4(0, 0, 0, 0);
+                       });
         return;
     }
     const long long work = S * cch;
@@ -1244,8 +1189,7 @@ ct_status dense_pair_run(const Plan &p, const void *x, const void *wp, const voi
         g.oz = -T.emin[0];
         g.oy = -T.emin[1];
         g.ox = -T.emin[2];
-        // about 8 halo stores per thread
-        g.halo_blocks = (int)std::max<long long>(1, std::min<long long>(1024, ceil_div(halo_count(g).n_all * 8, 2048)));
+        g.halo_blocks = halo_blocks_for(g);
         if (tiles + g.halo_blocks > 0x7fffffffLL || ceil_div(T.Cd, T.cpb) > 65535 || S >= (1LL << 31))
             return CT_ERR_UNSUPPORTED;
         dim3 grid((unsigned)(tiles + g.halo_blocks), (unsigned)ceil_div(T.Cd, T.cpb), (unsigned)T.N);
@@ -1253,7 +1197,7 @@ ct_status dense_pair_run(const Plan &p, const void *x, const void *wp, const voi
         if (T.nhwc) {
             // channels-last X: a padding copy of 16-byte pieces, about 8 per thread
             const long long pieces = (long long)T.C / (T.f32 ? 4 : 8);
-            g.halo_blocks = (int)std::max<long long>(1, std::min<long long>(1024, ceil_div(halo_count(g).n_all * pieces, 2048)));
+            g.halo_blocks = halo_blocks_for(g);
             const long long copy_blocks = std::max<long long>(1, std::min<long long>(8192, ceil_div(S * pieces, 2048)));
             dim3 gridc((unsigned)(g.halo_blocks + copy_blocks), 1, (unsigned)T.N);
             if (T.f32)
