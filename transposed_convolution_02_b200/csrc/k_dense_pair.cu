@@ -59,6 +59,14 @@ struct PItem {
     int16_t crow;     // first row of the item's half inside its chunk's half (either rank)
 };
 
+struct PadGeo {
+    int C, D, H, W;      // input extents
+    int Cd;              // channels of a padded position (C rounded up to a 16-byte row)
+    int HZ, HY, HX;      // padded extents
+    int oz, oy, ox;      // padded origin: zp = iz + oz, ...
+    int halo_blocks;     // blocks x = 0..halo_blocks-1 write the zero halo
+};
+
 struct PairTables {
     int32_t N, C, M, Np, KB;
     // f32: fp32 operands as a TF32 high part and its remainder (3xTF32: three
@@ -164,14 +172,6 @@ __global__ void __launch_bounds__(256) pair_prepack_kernel(const __grid_constant
 
 constexpr int kPadC = 64, kPadS = 128;
 
-struct PadGeo {
-    int C, D, H, W;      // input extents
-    int Cd;              // channels of a padded position (C rounded up to a 16-byte row)
-    int HZ, HY, HX;      // padded extents
-    int oz, oy, ox;      // padded origin: zp = iz + oz, ...
-    int halo_blocks;     // blocks x = 0..halo_blocks-1 write the zero halo
-};
-
 // Zero the halo of one image's padded copy, a padded row (zp, yp) at a time:
 // rows outside the input are zero for their whole width, the others only in
 // the columns left and right of the input.  Warp `wid` of `nw` takes rows
@@ -199,61 +199,77 @@ __device__ __forceinline__ void zero_halo_rows(const PadGeo &g, int wid, int nw,
     }
 }
 
-// Blocks that zero the halo: about one warp per padded row.
+// Blocks that zero the halo: about eight padded rows per warp (64 per block
+// of eight warps), so that halo and tile blocks together stay within one
+// wave of resident blocks for the workloads' sizes (a second, partial wave
+// measured as the re-layout's tail).
 inline int halo_blocks_for(const PadGeo &g) {
     const long long rows = (long long)g.HZ * g.HY;
-    return (int)std::max<long long>(1, std::min<long long>(256, ceil_div(rows, 8)));
+    return (int)std::max<long long>(1, std::min<long long>(256, ceil_div(rows, 64)));
 }
 
-__global__ void __launch_bounds__(256) nchw_to_padded_kernel(const __half *__restrict__ x,
-                                                             __half *__restrict__ xp, const PadGeo g) {
-    const int n = blockIdx.z;
-    const int C = g.C, Cd = g.Cd, H = g.H, W = g.W, HY = g.HY, HX = g.HX;
+// The padded re-layout of image n, one block of 256 threads per task (t is
+// the thread's index; `bar` the barrier the tile steps synchronise on, 0 for
+// the whole block): halo task h (0 <= h < halo_blocks) zeroes padded rows of
+// channel block cb; tile task st moves 64 channels x 128 input positions of
+// channel block cb through the 16 KB shared tile: its four 16-byte loads per
+// thread, then the 8x8-block transpose in shared memory and the stores.
+__device__ __forceinline__ void padded_halo(__half *__restrict__ xp, const PadGeo &g, int n, int cb, int halo, int t) {
+    const int Cd = g.Cd;
+    const long long P = (long long)g.HZ * g.HY * g.HX;
+    const int c0 = cb * kPadC;
+    const int c8 = (min(kPadC, Cd - c0)) >> 3;
+    __half *img = xp + (long long)n * P * Cd + c0;
+    zero_halo_rows(g, halo * 8 + (t >> 5), g.halo_blocks * 8, t & 31, c8,
+                   [&](long long pos, int q) {
+                       *reinterpret_cast<uint4 *>(img + pos * Cd + q * 8) = make_uint4(0, 0, 0, 0);
+                   });
+}
+
+__device__ __forceinline__ void padded_tile_load(const __half *__restrict__ x, const PadGeo &g, int n, int cb, int st,
+                                                 int t, uint4 (&v)[4]) {
+    const int C = g.C;
+    const long long S = (long long)g.D * g.H * g.W;
+    const int c0 = cb * kPadC;
+    const long long s0 = (long long)st * kPadS;
+    const bool vec = (S & 7) == 0;
+    const int cl = t >> 4, sv = t & 15;
+    const long long s = s0 + sv * 8;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const int c = c0 + cl + 16 * r;
+        const __half *src = x + ((long long)n * C + c) * S + s;
+        if (vec && c < C && s + 8 <= S) {
+            v[r] = __ldg(reinterpret_cast<const uint4 *>(src));
+        } else {
+            __align__(16) __half h[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) h[j] = (c < C && s + j < S) ? src[j] : __float2half(0.f);
+            v[r] = *reinterpret_cast<const uint4 *>(h);
+        }
+    }
+}
+
+__device__ __forceinline__ void padded_tile_finish(const uint4 (&v)[4], __half *__restrict__ xp, const PadGeo &g,
+                                                   int n, int cb, int st, __half *tile, int t, int bar) {
+    const int Cd = g.Cd, H = g.H, W = g.W, HY = g.HY, HX = g.HX;
     const long long HW = (long long)H * W;
     const long long S = g.D * HW;
     const long long P2 = (long long)HY * HX;
     const long long P = g.HZ * P2;
-    const int t = threadIdx.x;
-    sm100::griddep_launch_dependents();   // the pair kernel may set up while this one runs
-    if ((int)blockIdx.x < g.halo_blocks) {
-        // zero halo of image n, channels [c0, c0 + 64)
-        const int c0 = blockIdx.y * kPadC;
-        const int c8 = (min(kPadC, Cd - c0)) >> 3;
-        __half *img = xp + (long long)n * P * Cd + c0;
-        zero_halo_rows(g, (int)blockIdx.x * 8 + (t >> 5), g.halo_blocks * 8, t & 31, c8,
-                       [&](long long pos, int q) {
-                           *reinterpret_cast<uint4 *>(img + pos * Cd + q * 8) = make_uint4(0, 0, 0, 0);
-                       });
-        return;
-    }
-    __shared__ __align__(16) __half tile[kPadC][kPadS];
-    const int c0 = blockIdx.y * kPadC;
-    const long long s0 = (long long)(blockIdx.x - g.halo_blocks) * kPadS;
-    const bool vec = (S & 7) == 0;
+    const int c0 = cb * kPadC;
+    const long long s0 = (long long)st * kPadS;
     {
         const int cl = t >> 4, sv = t & 15;
-        const long long s = s0 + sv * 8;
-        uint4 v[4];
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            const int c = c0 + cl + 16 * r;
-            const __half *src = x + ((long long)n * C + c) * S + s;
-            if (vec && c < C && s + 8 <= S) {
-                v[r] = __ldg(reinterpret_cast<const uint4 *>(src));
-            } else {
-                __align__(16) __half h[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) h[j] = (c < C && s + j < S) ? src[j] : __float2half(0.f);
-                v[r] = *reinterpret_cast<const uint4 *>(h);
-            }
-        }
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
             const int row = cl + 16 * r;
-            *reinterpret_cast<uint4 *>(&tile[row][(sv ^ ((row >> 3) & 7)) * 8]) = v[r];
+            *reinterpret_cast<uint4 *>(tile + row * kPadS + ((sv ^ (row & 7)) * 8)) = v[r];
         }
     }
-    __syncthreads();
+    sm100::group_sync(bar);
+    // [64 channels][128 positions] -> [128 positions][64 channels], in place
+    sm100::transpose_64x128_b16(reinterpret_cast<uint16_t *>(tile), t >> 5, t & 31, bar);
     {
         const int sl = t >> 3, cv = t & 7;
         const int c = c0 + cv * 8;
@@ -278,14 +294,25 @@ __global__ void __launch_bounds__(256) nchw_to_padded_kernel(const __half *__res
             if (s >= S || c >= Cd) continue;   // channels C..Cd of the row are zeros
             const int zp = iz + g.oz, yp = iy + g.oy, xq = ix + g.ox;
             if (zp < 0 || zp >= g.HZ || yp < 0 || yp >= HY || xq < 0 || xq >= HX) continue;
-            __align__(16) __half v[8];
-            const int col = (((sp >> 3) ^ cv) << 3) | (sp & 7);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) v[j] = tile[cv * 8 + j][col];
             *reinterpret_cast<uint4 *>(xp + ((long long)n * P + zp * P2 + (long long)yp * HX + xq) * Cd + c) =
-                *reinterpret_cast<const uint4 *>(v);
+                *reinterpret_cast<const uint4 *>(tile + sp * 64 + ((cv ^ (sp & 7)) * 8));
         }
     }
+    sm100::group_sync(bar);   // the tile may be reused by the group's next task
+}
+
+__global__ void __launch_bounds__(256) nchw_to_padded_kernel(const __half *__restrict__ x,
+                                                             __half *__restrict__ xp, const PadGeo g) {
+    __shared__ __align__(128) __half tile[kPadC * kPadS];
+    sm100::griddep_launch_dependents();   // the pair kernel may set up while this one runs
+    if ((int)blockIdx.x < g.halo_blocks) {
+        padded_halo(xp, g, blockIdx.z, blockIdx.y, blockIdx.x, threadIdx.x);
+        return;
+    }
+    uint4 v[4];
+    const int st = (int)blockIdx.x - g.halo_blocks;
+    padded_tile_load(x, g, blockIdx.z, blockIdx.y, st, threadIdx.x, v);
+    padded_tile_finish(v, xp, g, blockIdx.z, blockIdx.y, st, tile, threadIdx.x, 0);
 }
 
 // fp32: X -> two padded channels-last planes, the TF32 high parts and the
@@ -434,7 +461,14 @@ __device__ __forceinline__ float act_f(float v) {
 __device__ __forceinline__ void st_pair(__half *p, float a, float b) {
     *reinterpret_cast<__half2 *>(p) = __floats2half2_rn(a, b);
 }
-__device__ __forceinline__ void st_pair(float *p, float a, float b) { *reinterpret_cast<float2 *>(p) = make_float2(a, b); }
+// fp32 outputs are written through to memory: with 3xTF32 the output stream
+// is far larger than L2 (the 1-D vocoder workload writes 268 MB), and
+// write-through keeps it from evicting the weight chunks that every unit
+// re-reads (measured: 665 -> 647 us per call on that workload; fp16 outputs,
+// which fit in L2 for the workloads, measured slower with it).
+__device__ __forceinline__ void st_pair(float *p, float a, float b) {
+    asm volatile("st.global.wt.v2.f32 [%0], {%1, %2};" ::"l"(p), "f"(a), "f"(b) : "memory");
+}
 __device__ __forceinline__ void st_one(__half *p, float a) { *p = __float2half_rn(a); }
 __device__ __forceinline__ void st_one(float *p, float a) { *p = a; }
 // 32 bias values from global memory (16-byte aligned source)

@@ -9,12 +9,12 @@ namespace {
 
 // channels-first -> channels-last re-layout of X (fp16), X[n][c][sp] -> Xt[n][sp][c].
 // A CTA moves a tile of 64 channels x 128 positions: every thread first
-// issues four 16-byte loads (four channel rows), then, after the exchange
-// through shared memory, four 16-byte stores (8 channels of one position
-// each), so each SM keeps many loads in flight and each position's 64
-// channels leave as one 128-byte run.  The 16-byte chunks of tile row r sit
-// at chunk index (chunk ^ (r >> 3) & 7), so the column reads of the eight
-// channel groups fall in distinct banks.
+// issues four 16-byte loads (four channel rows), the tile is transposed in
+// shared memory by 8x8 blocks (ldmatrix.trans, then stmatrix), and every
+// thread stores four 16-byte pieces (8 channels of one position each), so
+// each position's 64 channels leave as one 128-byte run.  Chunk q of tile
+// row r sits at chunk q ^ (r & 7) in both layouts, so the eight rows of an
+// 8x8 block fall in distinct banks.
 
 constexpr int kRlC = 64, kRlS = 128;
 
@@ -49,10 +49,13 @@ __global__ void __launch_bounds__(256) nchw_to_nhwc_kernel(const __half *__restr
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
             const int row = cl + 16 * r;
-            *reinterpret_cast<uint4 *>(&tile[row][(sv ^ ((row >> 3) & 7)) * 8]) = v[r];
+            *reinterpret_cast<uint4 *>(&tile[row][(sv ^ (row & 7)) * 8]) = v[r];
         }
     }
     __syncthreads();
+    // [64 channels][128 positions] -> [128 positions][64 channels], in place
+    sm100::transpose_64x128_b16(reinterpret_cast<uint16_t *>(&tile[0][0]), t >> 5, t & 31);
+    const __half *tout = &tile[0][0];
     {
         // 8 threads per position (8 x 8 channels), 32 positions per pass
         const int sl = t >> 3, cv = t & 7;
@@ -61,13 +64,9 @@ __global__ void __launch_bounds__(256) nchw_to_nhwc_kernel(const __half *__restr
         for (int r = 0; r < 4; ++r) {
             const int sp = sl + 32 * r;
             const long long s = s0 + sp;
-            if (s < S && c < C) {
-                __align__(16) __half v[8];
-                const int col = (((sp >> 3) ^ cv) << 3) | (sp & 7);   // rows cv*8 + j: (row >> 3) & 7 == cv
-#pragma unroll
-                for (int j = 0; j < 8; ++j) v[j] = tile[cv * 8 + j][col];
-                *reinterpret_cast<uint4 *>(xt + ((long long)n * S + s) * C + c) = *reinterpret_cast<const uint4 *>(v);
-            }
+            if (s < S && c < C)
+                *reinterpret_cast<uint4 *>(xt + ((long long)n * S + s) * C + c) =
+                    *reinterpret_cast<const uint4 *>(tout + sp * 64 + ((cv ^ (sp & 7)) * 8));
         }
     }
 }

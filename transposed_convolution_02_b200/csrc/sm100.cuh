@@ -172,6 +172,23 @@ __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// ---- 8x8 b16 matrix moves (shared memory <-> registers) ------------------------
+// Four 8x8 matrices of 16-bit elements: lanes 8i..8i+7 give the 16-byte row
+// addresses of matrix i, register i receives (or supplies) this thread's
+// fragment of matrix i (row lane/4, elements 2*(lane%4) and +1).  With
+// .trans the fragment is taken from the transposed matrix.
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t (&v)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3])
+                 : "r"(addr)
+                 : "memory");
+}
+__device__ __forceinline__ void stmatrix_x4(uint32_t addr, const uint32_t (&v)[4]) {
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v[0]), "r"(v[1]),
+                 "r"(v[2]), "r"(v[3])
+                 : "memory");
+}
+
 // One lane of the (fully active) warp gets true.
 __device__ __forceinline__ bool elect_one() {
     uint32_t pred = 0;
@@ -326,6 +343,45 @@ __host__ __device__ constexpr uint32_t idesc_tf32_f32(int M, int N) {
            | (0u << 15) | (0u << 16)    // A, B K-major
            | ((uint32_t)(N >> 3) << 17) // N / 8
            | ((uint32_t)(M >> 4) << 24);// M / 16
+}
+
+// Named barrier `id` over `count` threads (whole warps).
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+// Sync of the 256 threads that run a tile: the whole block (id 0), or the
+// named barrier `id` of a 256-thread group.
+__device__ __forceinline__ void group_sync(int id) {
+    if (id == 0)
+        __syncthreads();
+    else
+        named_bar_sync(id, 256);
+}
+
+// Transpose a tile of 64 rows x 128 16-bit elements (256-byte rows, 16-byte
+// chunk q of row r stored at chunk q ^ (r & 7)) in place into 128 rows x 64
+// elements (128-byte rows, chunk q of row r at q ^ (r & 7)), with 256
+// threads (warp 0..7 of the group synchronised by group_sync(bar_id)):
+// every warp moves sixteen 8x8 blocks, all reads before all writes.
+__device__ __forceinline__ void transpose_64x128_b16(uint16_t *tile, int warp, int lane, int bar_id = 0) {
+    uint32_t v[4][4];
+    const int mi = lane >> 3, r = lane & 7;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int blk = (warp * 4 + j) * 4 + mi;   // 8x8 block: 8 rows (cb) x 8 elements (pb)
+        const int cb = blk & 7, pb = blk >> 3;
+        const int row = cb * 8 + r;
+        ldmatrix_x4_trans(smem_u32(tile + row * 128 + ((pb ^ (row & 7)) * 8)), v[j]);
+    }
+    group_sync(bar_id);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int blk = (warp * 4 + j) * 4 + mi;
+        const int cb = blk & 7, pb = blk >> 3;
+        const int prow = pb * 8 + r;
+        stmatrix_x4(smem_u32(tile + prow * 64 + ((cb ^ (prow & 7)) * 8)), v[j]);
+    }
+    group_sync(bar_id);
 }
 
 }  // namespace sm100
