@@ -286,6 +286,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tmap(&tmA);
         prefetch_tmap(&tmB);
         if (rowmode) prefetch_tmap(&tmY);
+        // Start the first loads before the table copies and the TMEM
+        // allocation: the resident weights (the grid this one may overlap
+        // with, under programmatic launch, is the call's own re-layout or
+        // bias fill, which does not write them; see the launch), then, once
+        // that grid's output is visible, the first unit's input ring entries.
+        if (resident) {
+            mbar_arrive_expect_tx(bres, (uint32_t)res_rows * 128);
+            for (int r = 0; r < res_rows; r += BR) tma_load_2d(smem_u32(sB + (size_t)r * 128), &tmB, bres, 0, r);
+        }
+        griddep_wait();
+        if ((int)blockIdx.x < n_units) {
+            const Unit U = decode_unit(G, blockIdx.x);
+            const int x0 = U.tx * BXt + T.g_emin[U.g][2];
+            const int y0 = U.y0 + T.g_emin[U.g][1];
+            const int z0 = U.jz + T.g_emin[U.g][0];
+            const int pre = min(SA, KB * zslices);
+            for (int q = 0; q < pre; ++q) {
+                const int kb = q / zslices, z = q - kb * zslices;
+                mbar_arrive_expect_tx(fullA + 8 * q, a_bytes);
+                if (rowmode) {
+                    for (int e = 0; e < n_ex; ++e)
+                        tma_load_5d(smem_u32(sA + (size_t)q * a_stride + (size_t)e * box_rows * 128), &tmA,
+                                    fullA + 8 * q, kb * 64, x0 + e, y0, z0 + z, U.n);
+                } else {
+                    tma_load_5d(smem_u32(sA + (size_t)q * a_stride), &tmA, fullA + 8 * q, kb * 64, x0, y0, z0, U.n);
+                }
+            }
+        }
     }
     for (int i = threadIdx.x; i < n_items; i += kThreads) {
         SItem it;
@@ -318,8 +346,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         groups_s[g] = gr;
     }
     for (int i = threadIdx.x; i < 3 * n_phases; i += kThreads) phr_s[i] = T.phase_r[i / 3][i % 3];
-    for (int m = threadIdx.x; m < ((Np + 31) & ~31); m += kThreads)
-        bias_s[m] = (T.has_bias && m < M) ? __half2float(bias[m]) : 0.f;
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_slot), 512);
         tmem_relinquish();
@@ -331,8 +357,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == 0 && lane == 0) {
         // ---------------- input tiles ----------------
-        // X (or its channels-last copy) may be the previous grid's output
-        griddep_wait();
+        // (this thread issued the first unit's first ring entries above,
+        // after waiting for the grid whose output it reads)
+        const int pre = min(SA, KB * zslices);
         int ia = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
@@ -342,6 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int y0 = U.y0 + gr.emin[1];
             const int z0 = U.jz + gr.emin[0];
             for (int q = 0; q < KB * zslices && ok; ++q, ++ia) {
+                if (u == (int)blockIdx.x && q < pre) continue;   // issued in the set-up
                 const int kb = q / zslices, z = q - kb * zslices;
                 const int s = ia % SA;
                 if (ia >= SA && !mbar_wait(emptyA + 8 * s, ((ia / SA) - 1) & 1, err, 1)) {
@@ -364,14 +392,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if ((warp == 2 || warp == 3) && lane == 0) {
         // ---------------- weight tiles: two issuing warps, alternate ring items ----------------
         const int me = warp - 2;
-        griddep_wait();   // the packed weights may be the previous grid's output
-        if (resident) {
-            if (me == 0) {
-                mbar_arrive_expect_tx(bres, (uint32_t)res_rows * 128);
-                for (int r = 0; r < res_rows; r += BR) tma_load_2d(smem_u32(sB + (size_t)r * 128), &tmB, bres, 0, r);
-                mbar_wait(bres, 0, err, 3);
-            }
-        } else {
+        // resident weights: loaded in the set-up (the MMA warp waits for them)
+        if (!resident) {
+            griddep_wait();
             int ib = 0;
             bool ok = true;
             for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
@@ -595,6 +618,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else if (warp >= 4) {
         // ---------------- epilogue ----------------
+        // the bias, staged by the epilogue warps themselves (its global reads
+        // stay off the set-up's path to the first loads)
+        for (int m = (int)threadIdx.x - 128; m < ((Np + 31) & ~31); m += kThreads - 128)
+            bias_s[m] = (T.has_bias && m < M) ? __half2float(bias[m]) : 0.f;
+        named_bar_sync(1, kThreads - 128);
         const int lane_base = 32 * (warp & 3);   // the TMEM lane quarter this warp may read
         const int eh = (warp - 4) >> 2;           // first 32-channel chunk of this warp's set
         const int p = lane_base + lane;
@@ -1113,8 +1141,12 @@ ct_status dense_tc_run(const Plan &p, const void *x, const void *wp, const void 
     if (!(parts & CT_PART_MAIN)) return CT_OK;
     int grid = sm_count();
     if (grid > T.n_units) grid = T.n_units;
-    // programmatic dependent launch: the set-up overlaps the tail of the grid
-    // before; both producers wait for it before loading
+    // programmatic dependent launch when this call's own re-layout or bias
+    // fill runs just before: the set-up overlaps that grid's tail, and the
+    // kernel reads the packed weights before waiting for it (neither writes
+    // them; the grid before it is complete, as it was launched normally).
+    // Otherwise the kernel starts after all earlier work, like any launch.
+    const bool pdl = (parts & CT_PART_PREPARE) && (p.layout == CT_NCHW || T.dead);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid, 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
@@ -1124,7 +1156,7 @@ ct_status dense_tc_run(const Plan &p, const void *x, const void *wp, const void 
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = pdl ? 1 : 0;
     const __half *b = (const __half *)bias;
     __half *yy = (__half *)y;
     cudaError_t e;

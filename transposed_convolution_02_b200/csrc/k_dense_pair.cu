@@ -584,8 +584,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
         prefetch_tmap(&tmB);
         prefetch_tmap(&tmBs);
     }
-    for (int m = threadIdx.x; m < T.BL; m += kPThreads)
-        bias_s[m] = (T.has_bias && m < M) ? (float)bias[m] : 0.f;
     if (warp == 1) {
         tmem_alloc_pair(smem_u32(tmem_slot), 512);
         tmem_relinquish_pair();
@@ -747,6 +745,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
         mbar_wait(mdone, 0, err, 10);
     } else if (warp >= 4) {
         // ---------------- epilogue (both CTAs) ----------------
+        // the bias, staged by the epilogue warps themselves (its global reads
+        // stay off the set-up's path to the first loads)
+        for (int m = (int)threadIdx.x - 128; m < T.BL; m += kPThreads - 128)
+            bias_s[m] = (T.has_bias && m < M) ? (float)bias[m] : 0.f;
+        named_bar_sync(1, kPThreads - 128);
         const int lane_base = 32 * (warp & 3);   // the TMEM lane quarter this warp may read
         const int eh = (warp - 4) >> 2;           // which alternate chunks of channels
         const int p = lane_base + lane;
@@ -1128,7 +1131,7 @@ size_t pair_launch_smem(const PairTables &T) { return std::max<size_t>(pair_smem
 
 template <int ACT, typename E>
 ct_status launch_pair(const PairTables &T, const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmBs,
-                      const void *bias, void *y, cudaStream_t st) {
+                      const void *bias, void *y, bool pdl, cudaStream_t st) {
     static std::atomic<int> attr_set[64];
     if (!allow_smem(dense_pair_kernel<ACT, E>, attr_set, kPSmemBudget)) return CT_ERR_DEVICE;
     const size_t smem = pair_launch_smem(T);
@@ -1145,7 +1148,10 @@ ct_status launch_pair(const PairTables &T, const CUtensorMap &tmA, const CUtenso
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    // programmatic launch only right after this call's own re-layout: the
+    // weight loads start before the wait for that grid (it does not write
+    // them; the grids before it completed, as it was launched normally)
+    cfg.numAttrs = pdl ? 1 : 0;
     const E *b = (const E *)bias;
     E *yy = (E *)y;
     if (cudaLaunchKernelEx(&cfg, dense_pair_kernel<ACT, E>, tmA, tmB, tmBs, T, b, yy) != cudaSuccess) {
@@ -1284,12 +1290,13 @@ ct_status dense_pair_run(const Plan &p, const void *x, const void *wp, const voi
         if (s2 != CT_OK) return s2;
     }
     if (!(parts & CT_PART_MAIN)) return CT_OK;
+    const bool pdl = (parts & CT_PART_PREPARE) != 0;   // the re-layout runs just before
     if (T.f32) {
-        if (T.act == CT_ACT_RELU) return launch_pair<CT_ACT_RELU, float>(T, tmA, tmB, tmBs, bias, y, st);
-        return launch_pair<CT_ACT_IDENTITY, float>(T, tmA, tmB, tmBs, bias, y, st);
+        if (T.act == CT_ACT_RELU) return launch_pair<CT_ACT_RELU, float>(T, tmA, tmB, tmBs, bias, y, pdl, st);
+        return launch_pair<CT_ACT_IDENTITY, float>(T, tmA, tmB, tmBs, bias, y, pdl, st);
     }
-    if (T.act == CT_ACT_RELU) return launch_pair<CT_ACT_RELU, __half>(T, tmA, tmB, tmBs, bias, y, st);
-    return launch_pair<CT_ACT_IDENTITY, __half>(T, tmA, tmB, tmBs, bias, y, st);
+    if (T.act == CT_ACT_RELU) return launch_pair<CT_ACT_RELU, __half>(T, tmA, tmB, tmBs, bias, y, pdl, st);
+    return launch_pair<CT_ACT_IDENTITY, __half>(T, tmA, tmB, tmBs, bias, y, pdl, st);
 }
 
 int dense_pair_take_error(cudaStream_t st) { return take_error_word(g_dense_pair_err, st); }
