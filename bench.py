@@ -546,6 +546,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--plain", action="store_true",
                     help="profiling mode: eager ct_run launches of one workload, nothing else")
+    ap.add_argument("--sets", type=int, default=1,
+                    help="with --plain: X/Y buffer sets to rotate over (default 1)")
     ap.add_argument("--general", action="store_true",
                     help="time a set of general shapes (stride 1, 1x1, channels-last, many or few "
                          "channels) and print one JSON line per shape")
@@ -604,13 +606,15 @@ def main():
         device = torch.device("cuda", local)
         torch.cuda.set_device(device)
         op, x_cpu = build_op(wl, device)
-        x = x_cpu.to(device)
-        y = torch.empty(op.y_shape, dtype=wl.dtype, device=device)
-        for _ in range(args.warmup + args.steps):
-            op(x, out=y)
+        # --sets K > 1 rotates K X/Y buffer sets, so that a workload smaller
+        # than L2 still moves its data through DRAM as in the timed steps
+        xs = [x_cpu.to(device) for _ in range(args.sets)]
+        ys = [torch.empty(op.y_shape, dtype=wl.dtype, device=device) for _ in range(args.sets)]
+        for i in range(args.warmup + args.steps):
+            op(xs[i % args.sets], out=ys[i % args.sets])
         torch.cuda.synchronize(device)
         print(json.dumps({"plain": wl.name, "kernel": op.kernel, "launches": op.launches,
-                          "runs": args.warmup + args.steps}), flush=True)
+                          "runs": args.warmup + args.steps, "sets": args.sets}), flush=True)
         return
 
     dist_max = None
