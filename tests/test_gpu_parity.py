@@ -378,6 +378,46 @@ def test_grouped_one_phase_path(case):
     full_parity(case, torch.float16, 70, "nchw", algo="grouped", expect_kernel="grouped")
 
 
+@pytest.mark.parametrize("case", [
+    # many row blocks per CTA (16 images x 32 groups): the persistent CTAs
+    # walk several blocks each, with the tile of the next one in flight
+    dict(x_shape=[16, 512, 16, 16], w_shape=[512, 16, 3, 3], strides=[2, 2], dilations=[2, 2],
+         auto_pad="SAME_UPPER", group=32, bias=True),
+    # ragged last row block, the taps in the even phases (SAME_LOWER), ReLU
+    dict(x_shape=[3, 64, 21, 24], w_shape=[64, 16, 3, 3], strides=[2, 2], dilations=[2, 2],
+         auto_pad="SAME_LOWER", group=4, bias=True, activation="relu"),
+    # 64 channels per group (eight 8-channel pieces per pixel), 8 output channels
+    dict(x_shape=[2, 128, 10, 16], w_shape=[128, 8, 3, 3], strides=[2, 2], dilations=[2, 2],
+         auto_pad="SAME_UPPER", group=2, bias=True),
+    # rank 1 with a 256-wide output row, no bias
+    dict(x_shape=[4, 96, 128], w_shape=[96, 16, 3], strides=[2], dilations=[2],
+         auto_pad="SAME_UPPER", group=6, bias=False),
+    # stride 3 in y (two tap-less row phases), a 1x1 kernel (one tap),
+    # output_padding on both axes
+    dict(x_shape=[2, 32, 12, 16], w_shape=[32, 16, 1, 1], strides=[3, 2], pads=[0, 0, 0, 0],
+         output_padding=[2, 1], group=2, bias=True),
+])
+def test_grouped_stream_path(case):
+    """One-phase grouped shapes with 16-byte output rows (out_x % 8 == 0, at
+    most 256): the persistent form of the grouped kernel, whose tap-less rows
+    leave by TMA tensor stores of a bias tile.  Outputs that no tap reaches
+    must be exactly the activated bias; the rest within the fp16 tolerance."""
+    x, w, b = draw_case(case, torch.float16, 83)
+    op, y = gpu_run(case, x, w, b, "nchw", "grouped")
+    assert op.kernel == "grouped"
+    xa, wa, ba = to_oracle(x, w, b, "nchw")
+    act = case.get("activation", "identity")
+    ref, absacc = conv_transpose_ref(xa, wa, ba, attrs_from(case), activation=act)
+    check_close(y, ref, absacc, torch.float16, "%s grouped" % (case,))
+    bias_only = torch.from_numpy(absacc == 0)
+    assert bias_only.any()
+    bb = (b.float() if b is not None else torch.zeros(case["w_shape"][1] * case["group"]))
+    bb = (bb.clamp_min(0) if act == "relu" else bb).half()
+    want = bb.view([1, -1] + [1] * (y.dim() - 2)).expand(y.shape)
+    got = y.cpu()
+    assert torch.equal(got[bias_only], want[bias_only])
+
+
 @pytest.mark.parametrize("layout", ["nchw", "nhwc"])
 def test_fp32_gemm_random_sweep(layout):
     """fp32 group-1 shapes on the register-tiled FFMA phase GEMM: ranks 1-3,

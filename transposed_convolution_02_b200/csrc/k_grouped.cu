@@ -67,6 +67,12 @@ struct GroupedArgs {
     // shared-memory layout (byte offsets): input tile / staging union at 0, slab,
     // A fragments, step offsets, bias, barrier
     int32_t off_slab, off_w, off_steps, off_bias, off_bar, smem_total, raw_bytes, stage_bytes;
+    // streaming form of the one-phase path (grouped_stream_kernel): persistent
+    // CTAs, the input tile SRt x BW (channel stride an odd number of 16-byte
+    // units), bias tiles for the tap-less rows at off_btile (two of
+    // btile_bytes), the group's bias at off_sb (two of 64 halves)
+    int32_t stream, SRt, grid, off_btile, btile_bytes, off_sb, off_wst;
+    DivMagic d_qn, d_hn;
     DivMagic d_npix, d_sw, d_seg, d_lry, d_drow, d_segw, d_rb, d_g, d_cols, d_cprs, d_cprc;
     int8_t live_ry[kGMaxS], dead_ry[kGMaxS], live_rx[kGMaxS];
     uint8_t ph_q0[kGMaxS][kGMaxS], ph_nq[kGMaxS][kGMaxS];   // tap pairs of phase (ry, rx)
@@ -113,16 +119,17 @@ __device__ __forceinline__ uint32_t bias_word(__half b) {
 // swap half their words so that each lane stores 4 consecutive J of one
 // channel as one 16-byte piece (8-byte pieces when out_x % 8 != 0).
 template <int NSTEP, int ACT>
-__device__ __forceinline__ void one_phase_rows(const GroupedArgs &A, const uint4 *__restrict__ wp,
+__device__ __forceinline__ void one_phase_rows(const GroupedArgs &A, const uint4 *__restrict__ wp, uint32_t s_w,
                                                const __half *sb, uint32_t s_slab, __half *yg,
                                                long long plane, int g, int jy0, int jbv, int warp,
-                                               int lane) {
+                                               int lane, int nwarps) {
     const int gid = lane >> 2, tig = lane & 3;
     uint4 af[NSTEP];
     uint32_t offs[NSTEP];
 #pragma unroll
     for (int j = 0; j < NSTEP; ++j) {
-        af[j] = __ldg(wp + ((size_t)g * NSTEP + j) * 32 + lane);
+        // the group's fragments: staged in shared memory (s_w), else from global
+        af[j] = s_w ? lds_v4(s_w + 16 * (j * 32 + lane)) : __ldg(wp + ((size_t)g * NSTEP + j) * 32 + lane);
         offs[j] = (uint32_t)A.steps[j];
     }
     const int ry = A.live_ry[0], rx = A.live_rx[0];
@@ -146,7 +153,7 @@ __device__ __forceinline__ void one_phase_rows(const GroupedArgs &A, const uint4
     const int lpix = 8 * (lane >> 4) + (lane & 7);
     const uint32_t lrow = s_slab + 16 * ((lane >> 3) & 1);
     const int items = jbv * A.n_seg;
-    for (int it = warp; it < items; it += kGWarps) {
+    for (int it = warp; it < items; it += nwarps) {
         const int jyl = divq(it, A.d_seg);
         const int jx0 = (it - jyl * A.n_seg) * 16;
         const int oy = A.s_y * (jy0 + jyl) + ry;
@@ -338,7 +345,7 @@ __global__ void __launch_bounds__(kGThreads, NSTEP > 0 ? kGOnePhaseMinBlocks : (
     __syncthreads();
 
     if constexpr (NSTEP > 0) {
-        one_phase_rows<NSTEP, ACT>(A, wp, sb, s_slab, yg, plane, g, jy0, jbv, warp, lane);
+        one_phase_rows<NSTEP, ACT>(A, wp, 0u, sb, s_slab, yg, plane, g, jy0, jbv, warp, lane, kGWarps);
         return;
     }
     // staging tile (over the consumed input tile): every column starts as the
@@ -510,6 +517,137 @@ __global__ void __launch_bounds__(256) grouped_prepack_kernel(const __grid_const
     }
 }
 
+
+// The one-phase path as a persistent kernel.  CTA c walks blocks c, c +
+// gridDim.x, ... (neighbouring CTAs take neighbouring row blocks, so the
+// halo rows they share are read from DRAM once).  Warp 7 is the producer:
+//   * it loads each block's input tile and the group's weight fragments with
+//     TMA while the previous block is computed (one barrier for both; the
+//     fragments in two alternating buffers);
+//   * it stages the block's bias and a [Mg][out_x] tile of its activated
+//     value, and writes the block's tap-less output rows from that tile with
+//     TMA tensor stores (two tiles and bias buffers alternate; a tile is
+//     refilled only once the stores of two blocks back have read it).  It
+//     issues no global stores of its own, so its proxy fence before the bulk
+//     stores does not wait for the compute warps' outputs, and it prepares
+//     the next block's rows while the compute warps work on this one.
+// Per block, all warps re-lay the input tile channel-contiguous: each 8
+// channels x 8 pixels piece is read transposed with ldmatrix.trans and
+// written with stmatrix as 8 pixel rows of the slab (the tile's channel
+// stride is an odd number of 16-byte units, so the 8 rows of a piece fall in
+// distinct banks).  The tile is then free: the producer starts the next
+// load, and warps 0-6 compute the rows with taps as one_phase_rows does.
+template <int NSTEP, int ACT>
+__global__ void __launch_bounds__(kGThreads, kGOnePhaseMinBlocks)
+    grouped_stream_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmy,
+                          const __grid_constant__ GroupedArgs A, const uint4 *__restrict__ wp,
+                          const __half *__restrict__ bias, __half *__restrict__ y) {
+    extern __shared__ __align__(1024) uint8_t sm[];
+    constexpr int kProducer = kGWarps - 1;
+    constexpr uint32_t kWBytes = NSTEP * 512;   // one group's A fragments
+    const uint32_t s0 = smem_u32(sm);
+    const uint32_t s_tile = s0;
+    const uint32_t s_slab = s0 + A.off_slab;
+    const uint32_t s_btile = s0 + A.off_btile;
+    const uint32_t s_wst = s0 + A.off_wst;
+    const uint32_t bar = s0 + A.off_bar;
+    const uint32_t s_sink = bar + 16;   // 16 bytes that absorb the pixels outside the slab
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int n_blocks = A.N * A.G * A.n_rb;
+    const long long plane = (long long)A.out_y * A.out_x;
+    const uint32_t cs = (uint32_t)A.SRt * A.BW * 2;   // channel stride of the tile, bytes
+    const int qn = A.BW >> 3, hn = A.Cg >> 3;
+    const int pieces = A.SR * qn * hn;                 // 8 x 8 pieces of the slab's rows
+    const bool loader = warp == kProducer && lane == 0;
+
+    auto coords = [&](int b, int &n, int &g, int &jy0) {
+        const int bq = divq(b, A.d_rb);
+        n = divq(bq, A.d_g);
+        g = bq - n * A.G;
+        jy0 = (b - bq * A.n_rb) * A.JB;
+    };
+    // the tile and the fragments of block b (its k-th) on the barrier
+    auto load_block = [&](int b, int k) {
+        int n, g, jy0;
+        coords(b, n, g, jy0);
+        mbar_arrive_expect_tx(bar, (uint32_t)A.raw_bytes + kWBytes);
+        tma_load_3d(s_tile, &tmx, bar, A.x0, jy0 + A.emin_y, n * A.C + g * A.Cg);
+        bulk_load(s_wst + (uint32_t)(k & 1) * kWBytes, wp + (size_t)g * NSTEP * 32, kWBytes, bar);
+    };
+    if (loader) {
+        mbar_init(bar, 1);
+        fence_barrier_init();
+        prefetch_tmap(&tmx);
+        prefetch_tmap(&tmy);
+        if ((int)blockIdx.x < n_blocks) load_block(blockIdx.x, 0);
+    }
+    __syncthreads();
+
+    int k = 0;
+    bool ok = true;
+    for (int b = blockIdx.x; b < n_blocks; b += gridDim.x, ++k) {
+        int n, g, jy0;
+        coords(b, n, g, jy0);
+        const int jbv = min(A.JB, A.nJy - jy0);
+        __half *sb = reinterpret_cast<__half *>(sm + A.off_sb) + 64 * (k & 1);
+        if (warp == kProducer) {
+            sb[lane] = (A.has_bias && lane < A.Mg) ? bias[g * A.Mg + lane] : __float2half(0.f);
+            sb[lane + 32] = (A.has_bias && lane + 32 < A.Mg) ? bias[g * A.Mg + lane + 32] : __float2half(0.f);
+            if (A.n_dead_ry > 0) {
+                const uint32_t bt = s_btile + (uint32_t)(k & 1) * A.btile_bytes;
+                if (lane == 0) bulk_wait_group_read<1>();   // the stores of block k - 2 have read this tile
+                __syncwarp();
+                const int cpr = A.out_x >> 3;   // 16-byte pieces per channel row
+                for (int e = lane; e < A.Mg * cpr; e += 32) {
+                    const int m = divq(e, A.d_cols);
+                    const uint32_t w = bias_word(__float2half_rn(apply_act(__half2float(sb[m]), ACT)));
+                    sts_v4(bt + 16 * e, make_uint4(w, w, w, w));
+                }
+                fence_proxy_async();   // the tile, written here, before the bulk stores read it
+                __syncwarp();
+                if (lane == 0) {
+                    for (int jyl = 0; jyl < jbv; ++jyl)
+                        for (int d = 0; d < A.n_dead_ry; ++d) {
+                            const int oy = A.s_y * (jy0 + jyl) + A.dead_ry[d];
+                            if (oy < A.out_y) tma_store_3d(&tmy, bt, 0, oy, n * A.M + g * A.Mg);
+                        }
+                    bulk_commit_group();
+                }
+            }
+        }
+        // the block's input tile and fragments; every compute warp has finished the previous block
+        ok = mbar_wait(bar, k & 1, &g_grouped_err, 2);
+        if (!__syncthreads_and(ok)) break;
+        {
+            const int i = lane & 7, sub = lane >> 3;
+            for (int o = 4 * warp; o < pieces; o += 4 * kGWarps) {
+                const int pc = min(o + sub, pieces - 1);
+                const int t = divq(pc, A.d_qn);   // piece = (r * hn + h) * qn + q
+                const int q = pc - t * qn;
+                const int r = divq(t, A.d_hn);
+                const int h = t - r * hn;
+                uint32_t v[4];
+                ldmatrix_x4_trans(s_tile + (uint32_t)(8 * h + i) * cs + (uint32_t)(r * A.BW + 8 * q) * 2, v);
+                const int c = 8 * q + i - A.dx;   // slab column of this lane's pixel row
+                const uint32_t dst = (c >= 0 && c < A.SW) ? s_slab + (uint32_t)(r * A.SW + c) * A.pst + 16 * h : s_sink;
+                stmatrix_x4(dst, v);
+            }
+        }
+        __syncthreads();   // slab complete, tile consumed
+        if (warp == kProducer) {
+            if (lane == 0 && b + (int)gridDim.x < n_blocks) {
+                fence_proxy_async();
+                load_block(b + (int)gridDim.x, k + 1);
+            }
+        } else {
+            __half *yg = y + ((long long)n * A.M + (long long)g * A.Mg) * plane;
+            one_phase_rows<NSTEP, ACT>(A, wp, s_wst + (uint32_t)(k & 1) * kWBytes, sb, s_slab, yg, plane, g, jy0,
+                                       jbv, warp, lane, kProducer);
+        }
+    }
+    if (!ok && loader) mbar_wait(bar, k & 1, &g_grouped_err, 3);   // the load that timed out, drained
+    if (loader) bulk_wait_group_all();
+}
 }  // namespace
 
 bool grouped_setup(const Plan &p, GroupedArgs &A, int jb);
@@ -682,9 +820,102 @@ size_t grouped_packed_bytes(const Plan &p) {
     return (size_t)A.G * A.n_pairs * A.KS * A.MT * 32 * 16;
 }
 
+// CTAs of grouped_stream_kernel<NSTEP> resident per SM with `smem` bytes of
+// shared memory (the occupancy calculator when a device answers, else the
+// launch bound and the shared-memory capacity).
+template <int NSTEP>
+int stream_blocks_per_sm_n(int smem) {
+    static std::atomic<int> attr_set[64];
+    int n = 0;
+    if (allow_smem(grouped_stream_kernel<NSTEP, CT_ACT_IDENTITY>, attr_set, kGSmem) &&
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, grouped_stream_kernel<NSTEP, CT_ACT_IDENTITY>, kGThreads,
+                                                      (size_t)smem) == cudaSuccess &&
+        n > 0)
+        return n;
+    cudaGetLastError();
+    return std::min(kGOnePhaseMinBlocks, (228 * 1024) / (smem + 1024));
+}
+
+int stream_blocks_per_sm(int nstep, int smem) {
+    switch (nstep) {
+        case 1: return stream_blocks_per_sm_n<1>(smem);
+        case 2: return stream_blocks_per_sm_n<2>(smem);
+        case 3: return stream_blocks_per_sm_n<3>(smem);
+        case 4: return stream_blocks_per_sm_n<4>(smem);
+        case 6: return stream_blocks_per_sm_n<6>(smem);
+        case 8: return stream_blocks_per_sm_n<8>(smem);
+        case 9: return stream_blocks_per_sm_n<9>(smem);
+        case 12: return stream_blocks_per_sm_n<12>(smem);
+    }
+    return 0;
+}
+
+// The streaming form of the one-phase path for J-row blocks of `jb` rows:
+// the input tile widened so that its channel stride is an odd number of
+// 16-byte units (SRt rows, BW columns, both giving an odd count), the bias
+// tiles and the shared-memory layout.  False when the shape or the block
+// does not suit it.
+bool stream_setup(const Plan &p, GroupedArgs &A, int jb) {
+    if (!grouped_setup(p, A, jb)) return false;
+    if (!A.one_phase || !A.use_tma || !A.vec8 || A.out_x > 256 || A.Mg > 64) return false;
+    if ((long long)A.N * A.M >= (1LL << 31) || (long long)A.N * A.C >= (1LL << 31)) return false;
+    if ((A.BW / 8) % 2 == 0) A.BW += 8;
+    A.SRt = A.SR | 1;
+    if (A.BW > 256 || A.SRt > 256) return false;
+    A.raw_bytes = A.Cg * A.SRt * A.BW * 2;
+    A.btile_bytes = A.n_dead_ry > 0 ? (int32_t)round_up((size_t)A.Mg * A.out_x * 2, 128) : 0;
+    const size_t tile = round_up((size_t)A.raw_bytes, 128);
+    const size_t slab = round_up((size_t)A.npix * A.pst, 128);
+    A.off_slab = (int32_t)tile;
+    A.off_btile = (int32_t)(tile + slab);
+    A.off_wst = A.off_btile + 2 * A.btile_bytes;
+    A.off_sb = A.off_wst + 2 * A.one_phase * 512;
+    A.off_bar = A.off_sb + 2 * 64 * 2;
+    A.smem_total = A.off_bar + 32;   // barrier, then a 16-byte sink for pixels outside the slab
+    if (A.smem_total > kGSmem) return false;
+    A.d_qn = make_magic((uint32_t)(A.BW / 8));
+    A.d_hn = make_magic((uint32_t)(A.Cg / 8));
+    A.stream = 1;
+    return true;
+}
+
+// Pick the streaming form's J-row block: among blocks whose shared memory
+// leaves kGOnePhaseMinBlocks CTAs per SM, the fewest rounds of the grid
+// times the rows a block computes plus two (the halo and per-block set-up
+// in row units).
+bool stream_plan(const Plan &p, GroupedArgs &A) {
+    const long long sms = sm_count();
+    long long best_cost = -1;
+    int best_jb = 0, best_per_sm = 0;
+    for (int jb = 2; jb <= 32; ++jb) {
+        GroupedArgs T;
+        if (!stream_setup(p, T, jb)) continue;
+        const int per_sm = stream_blocks_per_sm(T.one_phase, T.smem_total);
+        if (per_sm < kGOnePhaseMinBlocks) continue;
+        const long long slots = (long long)per_sm * sms;
+        const long long blocks = (long long)T.N * T.G * T.n_rb;
+        const long long cost = ceil_div(blocks, slots) * (T.JB + 2);
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best_jb = jb;
+            best_per_sm = per_sm;
+        }
+        if (T.JB >= T.nJy) break;
+    }
+    if (best_cost < 0 || !stream_setup(p, A, best_jb)) return false;
+    const long long blocks = (long long)A.N * A.G * A.n_rb;
+    if (blocks > 0x7fffffffLL) return false;
+    A.grid = (int32_t)std::min<long long>(blocks, (long long)best_per_sm * sms);
+    return true;
+}
+
 void grouped_plan(Plan &p) {
     p.aux.assign((sizeof(GroupedArgs) + 7) / 8, 0);
     GroupedArgs &A = *reinterpret_cast<GroupedArgs *>(p.aux.data());
+    if (stream_plan(p, A)) {
+        p.launches = 1;
+        return;
+    }
     // J rows per CTA: the largest power of two whose shared memory stays
     // within 56 KB (four CTAs per SM) while the grid still gives every SM
     // a dozen CTAs; one row at least.
@@ -728,9 +959,70 @@ ct_status launch_grouped(const CUtensorMap &tm, const GroupedArgs &A, const void
     return launch_grouped_act<MT, NSTEP, CT_ACT_IDENTITY>(tm, A, x, wp, bias, y, grid, st);
 }
 
+template <int NSTEP, int ACT>
+ct_status launch_stream_act(const CUtensorMap &tmx, const CUtensorMap &tmy, const GroupedArgs &A, const void *wp,
+                            const void *bias, void *y, cudaStream_t st) {
+    static std::atomic<int> attr_set[64];
+    if (!allow_smem(grouped_stream_kernel<NSTEP, ACT>, attr_set, kGSmem)) return CT_ERR_DEVICE;
+    grouped_stream_kernel<NSTEP, ACT><<<(unsigned)A.grid, kGThreads, (size_t)A.smem_total, st>>>(
+        tmx, tmy, A, (const uint4 *)wp, (const __half *)bias, (__half *)y);
+    return launch_status();
+}
+
+template <int NSTEP>
+ct_status launch_stream(const CUtensorMap &tmx, const CUtensorMap &tmy, const GroupedArgs &A, const void *wp,
+                        const void *bias, void *y, cudaStream_t st) {
+    if (A.act == CT_ACT_RELU) return launch_stream_act<NSTEP, CT_ACT_RELU>(tmx, tmy, A, wp, bias, y, st);
+    return launch_stream_act<NSTEP, CT_ACT_IDENTITY>(tmx, tmy, A, wp, bias, y, st);
+}
+
+ct_status grouped_stream_run(const GroupedArgs &A, const void *x, const void *wp, const void *bias, void *y,
+                             cudaStream_t st) {
+    if (A.grid <= 0) return CT_OK;
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return CT_ERR_DEVICE;
+    CUtensorMap tmx, tmy;
+    memset(&tmx, 0, sizeof(tmx));
+    memset(&tmy, 0, sizeof(tmy));
+    {
+        // X as (x, y, image * channel); the box is one block's input tile
+        const cuuint64_t dims[3] = {(cuuint64_t)A.in_x, (cuuint64_t)A.in_y, (cuuint64_t)A.N * A.C};
+        const cuuint64_t strides[2] = {(cuuint64_t)A.in_x * 2, (cuuint64_t)A.in_x * A.in_y * 2};
+        const cuuint32_t box[3] = {(cuuint32_t)A.BW, (cuuint32_t)A.SRt, (cuuint32_t)A.Cg};
+        const cuuint32_t es[3] = {1, 1, 1};
+        if (enc(&tmx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void *>(x), dims, strides, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return CT_ERR_DEVICE;
+    }
+    {
+        // Y as (x, y, image * channel); the box is one output row of a group's channels
+        const cuuint64_t dims[3] = {(cuuint64_t)A.out_x, (cuuint64_t)A.out_y, (cuuint64_t)A.N * A.M};
+        const cuuint64_t strides[2] = {(cuuint64_t)A.out_x * 2, (cuuint64_t)A.out_x * A.out_y * 2};
+        const cuuint32_t box[3] = {(cuuint32_t)A.out_x, 1, (cuuint32_t)A.Mg};
+        const cuuint32_t es[3] = {1, 1, 1};
+        if (enc(&tmy, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, y, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return CT_ERR_DEVICE;
+    }
+    switch (A.one_phase) {
+        case 1: return launch_stream<1>(tmx, tmy, A, wp, bias, y, st);
+        case 2: return launch_stream<2>(tmx, tmy, A, wp, bias, y, st);
+        case 3: return launch_stream<3>(tmx, tmy, A, wp, bias, y, st);
+        case 4: return launch_stream<4>(tmx, tmy, A, wp, bias, y, st);
+        case 6: return launch_stream<6>(tmx, tmy, A, wp, bias, y, st);
+        case 8: return launch_stream<8>(tmx, tmy, A, wp, bias, y, st);
+        case 9: return launch_stream<9>(tmx, tmy, A, wp, bias, y, st);
+        case 12: return launch_stream<12>(tmx, tmy, A, wp, bias, y, st);
+    }
+    return CT_ERR_UNSUPPORTED;
+}
+
 ct_status grouped_run(const Plan &p, const void *x, const void *wp, const void *bias, void *y,
                       cudaStream_t st) {
     const GroupedArgs &A = gargs(p);
+    if (A.stream) return grouped_stream_run(A, x, wp, bias, y, st);
     if (A.smem_total > kGSmem) return CT_ERR_UNSUPPORTED;
     const long long grid = (long long)A.N * A.G * A.n_rb;
     if (grid > 0x7fffffffLL) return CT_ERR_UNSUPPORTED;

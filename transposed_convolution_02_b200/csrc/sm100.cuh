@@ -103,6 +103,12 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_
 // box) is written to the box at the given coordinates; parts of the box
 // outside the tensor are not written.  Threads that wrote the tile must
 // execute fence_proxy_async() before the issuing thread starts the store.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, uint32_t src, int32_t c0, int32_t c1,
+                                             int32_t c2) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(map),
+                 "r"(src), "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
+}
 __device__ __forceinline__ void tma_store_5d(const CUtensorMap *map, uint32_t src, int32_t c0, int32_t c1,
                                              int32_t c2, int32_t c3, int32_t c4) {
     asm volatile(
