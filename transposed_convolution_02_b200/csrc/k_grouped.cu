@@ -113,11 +113,12 @@ __device__ __forceinline__ uint32_t bias_word(__half b) {
 }
 
 // Segments of the one-phase path: outputs o = 2*J + rx of row oy, channel m,
-// get bias (other column phase) and value in one 32-bit word per J.  The
-// weight fragments (A operand) stay in registers for the whole CTA; B
-// fragments are loaded two steps ahead of the MMAs that use them.  Lane pairs
-// swap half their words so that each lane stores 4 consecutive J of one
-// channel as one 16-byte piece (8-byte pieces when out_x % 8 != 0).
+// get bias (other column phase) and value in one 32-bit word per J, packed by
+// one f32x2 -> f16x2 conversion.  The weight fragments (A operand) stay in
+// registers for the whole CTA; B fragments are loaded two steps ahead of the
+// MMAs that use them.  Each lane stores its two J of channels gid and gid + 8
+// as two 8-byte pieces: the four lanes of a channel row write 32 contiguous
+// bytes, a whole sector.
 template <int NSTEP, int ACT>
 __device__ __forceinline__ void one_phase_rows(const GroupedArgs &A, const uint4 *__restrict__ wp, uint32_t s_w,
                                                const __half *sb, uint32_t s_slab, __half *yg,
@@ -135,17 +136,9 @@ __device__ __forceinline__ void one_phase_rows(const GroupedArgs &A, const uint4
     const int ry = A.live_ry[0], rx = A.live_rx[0];
     const __half b0h = sb[gid], b1h = sb[gid + 8];
     const float bf0 = __half2float(b0h), bf1 = __half2float(b1h);
-    // the other column phase's outputs: activated bias
-    const uint32_t bw0 = __half_as_ushort(__float2half_rn(apply_act(bf0, ACT)));
-    const uint32_t bw1 = __half_as_ushort(__float2half_rn(apply_act(bf1, ACT)));
-    // (bias, value) order inside a 32-bit word: value high when rx == 1
-    const int vsh = rx ? 16 : 0, bsh = rx ? 0 : 16;
-    const bool odd = tig & 1;
-    // 16-byte pieces: an even lane stores channel gid, J = 2*tig + [0, 4); an
-    // odd lane channel gid + 8, J = 2*(tig - 1) + [0, 4)
-    const int mv = gid + (odd ? 8 : 0);
-    const bool okv = mv < A.Mg;
-    __half *yv = yg + (long long)mv * plane + 4 * (tig & 2);
+    // the other column phase's outputs: activated bias (exact in fp16)
+    const float bo0 = __half2float(__float2half_rn(apply_act(bf0, ACT)));
+    const float bo1 = __half2float(__float2half_rn(apply_act(bf1, ACT)));
     // 8-byte pieces: channels gid and gid + 8, J = 2*tig + [0, 2)
     const bool ok0 = gid < A.Mg, ok1 = gid + 8 < A.Mg;
     __half *y0 = yg + (long long)gid * plane + 4 * tig;
@@ -188,32 +181,23 @@ __device__ __forceinline__ void one_phase_rows(const GroupedArgs &A, const uint4
                 : "+f"(acc[1][0]), "+f"(acc[1][1]), "+f"(acc[1][2]), "+f"(acc[1][3])
                 : "r"(af[j].x), "r"(af[j].y), "r"(af[j].z), "r"(af[j].w), "r"(b[2]), "r"(b[3]));
         }
-        // words: channel gid at J = jx0 + 8*nt + 2*tig + {0,1} (w[nt][0..1]),
-        // channel gid + 8 (w[nt][2..3]); nJx is even (out_x % 4 == 0), so each
-        // J pair lies inside the row or wholly past it
+        // words: channel gid at J = jx0 + 8*nt + 2*tig + {0,1} (acc[nt][0..1]),
+        // channel gid + 8 (acc[nt][2..3]); (bias, value) order inside a word:
+        // value high when rx == 1.  nJx is even (out_x % 4 == 0), so each J
+        // pair lies inside the row or wholly past it.
         const long long rowoff = (long long)oy * A.out_x + 2 * jx0;
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
+            if (jx0 + 8 * nt + 2 * tig >= A.nJx) continue;
             uint32_t w[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-                w[i] = ((uint32_t)__half_as_ushort(__float2half_rn(apply_act(acc[nt][i], ACT))) << vsh) |
-                       ((i < 2 ? bw0 : bw1) << bsh);
-            const int jx = jx0 + 8 * nt + 2 * tig;
-            if (A.vec8) {
-                // even lane keeps channel gid and takes the partner's channel-gid
-                // pair; odd lane keeps channel gid + 8 and takes the partner's
-                const uint32_t s0 = __shfl_xor_sync(0xffffffffu, odd ? w[0] : w[2], 1);
-                const uint32_t s1 = __shfl_xor_sync(0xffffffffu, odd ? w[1] : w[3], 1);
-                const int jv = jx0 + 8 * nt + 2 * (tig & 2);   // first J of this lane's piece
-                if (okv && jv < A.nJx) {
-                    const uint4 v = odd ? make_uint4(s0, s1, w[2], w[3]) : make_uint4(w[0], w[1], s0, s1);
-                    *reinterpret_cast<uint4 *>(yv + rowoff + 16 * nt) = v;
-                }
-            } else if (jx < A.nJx) {
-                if (ok0) *reinterpret_cast<uint2 *>(y0 + rowoff + 16 * nt) = make_uint2(w[0], w[1]);
-                if (ok1) *reinterpret_cast<uint2 *>(y1 + rowoff + 16 * nt) = make_uint2(w[2], w[3]);
+            for (int i = 0; i < 4; ++i) {
+                const float v = apply_act(acc[nt][i], ACT), o = i < 2 ? bo0 : bo1;
+                const __half2 h2 = rx ? __floats2half2_rn(o, v) : __floats2half2_rn(v, o);
+                w[i] = *reinterpret_cast<const uint32_t *>(&h2);
             }
+            if (ok0) *reinterpret_cast<uint2 *>(y0 + rowoff + 16 * nt) = make_uint2(w[0], w[1]);
+            if (ok1) *reinterpret_cast<uint2 *>(y1 + rowoff + 16 * nt) = make_uint2(w[2], w[3]);
         }
     }
 }
