@@ -71,8 +71,8 @@ struct GroupedArgs {
     // CTAs, the input tile SRt x BW (channel stride an odd number of 16-byte
     // units), bias tiles for the tap-less rows at off_btile (two of
     // btile_bytes), the group's bias at off_sb (two of 64 halves)
-    int32_t stream, SRt, grid, off_btile, btile_bytes, off_sb, off_wst;
-    DivMagic d_qn, d_hn;
+    int32_t stream, SRt, grid, off_btile, btile_bytes, off_sb, off_wst, n_seg32;
+    DivMagic d_qn, d_hn, d_seg32;
     DivMagic d_npix, d_sw, d_seg, d_lry, d_drow, d_segw, d_rb, d_g, d_cols, d_cprs, d_cprc;
     int8_t live_ry[kGMaxS], dead_ry[kGMaxS], live_rx[kGMaxS];
     uint8_t ph_q0[kGMaxS][kGMaxS], ph_nq[kGMaxS][kGMaxS];   // tap pairs of phase (ry, rx)
@@ -188,6 +188,84 @@ __device__ __forceinline__ void one_phase_rows(const GroupedArgs &A, const uint4
         const long long rowoff = (long long)oy * A.out_x + 2 * jx0;
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
+            if (jx0 + 8 * nt + 2 * tig >= A.nJx) continue;
+            uint32_t w[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float v = apply_act(acc[nt][i], ACT), o = i < 2 ? bo0 : bo1;
+                const __half2 h2 = rx ? __floats2half2_rn(o, v) : __floats2half2_rn(v, o);
+                w[i] = *reinterpret_cast<const uint32_t *>(&h2);
+            }
+            if (ok0) *reinterpret_cast<uint2 *>(y0 + rowoff + 16 * nt) = make_uint2(w[0], w[1]);
+            if (ok1) *reinterpret_cast<uint2 *>(y1 + rowoff + 16 * nt) = make_uint2(w[2], w[3]);
+        }
+    }
+}
+
+// one_phase_rows for the persistent kernel: items of 32 J (four n-tiles of
+// 8) whose MMAs share each step's weight fragment, read from shared memory
+// (s_w) once per step, so the per-item work (position decode, accumulator
+// set-up, loop) is spread over twice the outputs and the four accumulator
+// chains hide each other's MMA latency.  B fragments are loaded one step
+// ahead.  Stores as one_phase_rows does.
+template <int NSTEP, int ACT>
+__device__ __forceinline__ void one_phase_rows32(const GroupedArgs &A, uint32_t s_w, const __half *sb,
+                                                 uint32_t s_slab, __half *yg, long long plane, int jy0, int jbv,
+                                                 int warp, int lane, int nwarps) {
+    const int gid = lane >> 2, tig = lane & 3;
+    const int ry = A.live_ry[0], rx = A.live_rx[0];
+    const float bf0 = __half2float(sb[gid]), bf1 = __half2float(sb[gid + 8]);
+    // the other column phase's outputs: activated bias (exact in fp16)
+    const float bo0 = __half2float(__float2half_rn(apply_act(bf0, ACT)));
+    const float bo1 = __half2float(__float2half_rn(apply_act(bf1, ACT)));
+    const bool ok0 = gid < A.Mg, ok1 = gid + 8 < A.Mg;
+    __half *y0 = yg + (long long)gid * plane + 4 * tig;
+    __half *y1 = y0 + 8 * plane;
+    const int lpix = 8 * (lane >> 4) + (lane & 7);
+    const uint32_t lrow = s_slab + 16 * ((lane >> 3) & 1);
+    const uint32_t aw = s_w + 16 * lane;   // this lane's A fragment of step j at aw + 512 * j
+    const int items = jbv * A.n_seg32;
+    for (int it = warp; it < items; it += nwarps) {
+        const int jyl = divq(it, A.d_seg32);
+        const int jx0 = (it - jyl * A.n_seg32) * 32;
+        const int oy = A.s_y * (jy0 + jyl) + ry;
+        if (oy >= A.out_y) continue;
+        const uint32_t rowb = lrow + (uint32_t)(jyl * A.SW) * A.pst;
+        const uint32_t lb0 = rowb + (uint32_t)min(jx0 + lpix, A.nJx - 1) * A.pst;
+        const uint32_t lb1 = rowb + (uint32_t)min(jx0 + 16 + lpix, A.nJx - 1) * A.pst;
+        float acc[4][4];
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) {
+            acc[nt][0] = acc[nt][1] = bf0;
+            acc[nt][2] = acc[nt][3] = bf1;
+        }
+        uint32_t bq[2][8];
+        auto load_b = [&](int j, uint32_t(&b)[8]) {
+            const uint32_t o = (uint32_t)A.steps[j];
+            asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                         : "=r"(b[0]), "=r"(b[1]), "=r"(b[2]), "=r"(b[3])
+                         : "r"(lb0 + o));
+            asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                         : "=r"(b[4]), "=r"(b[5]), "=r"(b[6]), "=r"(b[7])
+                         : "r"(lb1 + o));
+        };
+        load_b(0, bq[0]);
+#pragma unroll
+        for (int j = 0; j < NSTEP; ++j) {
+            if (j + 1 < NSTEP) load_b(j + 1, bq[(j + 1) & 1]);
+            const uint32_t(&b)[8] = bq[j & 1];
+            const uint4 a = lds_v4(aw + 512 * j);
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+                asm volatile(
+                    "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+                    "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+                    : "+f"(acc[nt][0]), "+f"(acc[nt][1]), "+f"(acc[nt][2]), "+f"(acc[nt][3])
+                    : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b[2 * nt]), "r"(b[2 * nt + 1]));
+        }
+        const long long rowoff = (long long)oy * A.out_x + 2 * jx0;
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) {
             if (jx0 + 8 * nt + 2 * tig >= A.nJx) continue;
             uint32_t w[4];
 #pragma unroll
@@ -625,8 +703,8 @@ __global__ void __launch_bounds__(kGThreads, kGOnePhaseMinBlocks)
             }
         } else {
             __half *yg = y + ((long long)n * A.M + (long long)g * A.Mg) * plane;
-            one_phase_rows<NSTEP, ACT>(A, wp, s_wst + (uint32_t)(k & 1) * kWBytes, sb, s_slab, yg, plane, g, jy0,
-                                       jbv, warp, lane, kProducer);
+            one_phase_rows32<NSTEP, ACT>(A, s_wst + (uint32_t)(k & 1) * kWBytes, sb, s_slab, yg, plane, jy0, jbv,
+                                         warp, lane, kProducer);
         }
     }
     if (!ok && loader) mbar_wait(bar, k & 1, &g_grouped_err, 3);   // the load that timed out, drained
@@ -859,14 +937,16 @@ bool stream_setup(const Plan &p, GroupedArgs &A, int jb) {
     if (A.smem_total > kGSmem) return false;
     A.d_qn = make_magic((uint32_t)(A.BW / 8));
     A.d_hn = make_magic((uint32_t)(A.Cg / 8));
+    A.n_seg32 = (A.nJx + 31) / 32;
+    A.d_seg32 = make_magic((uint32_t)A.n_seg32);
     A.stream = 1;
     return true;
 }
 
 // Pick the streaming form's J-row block: among blocks whose shared memory
 // leaves kGOnePhaseMinBlocks CTAs per SM, the fewest rounds of the grid
-// times the rows a block computes plus two (the halo and per-block set-up
-// in row units).
+// times the 32-J items each compute warp takes per block plus one (the
+// re-layout and per-block set-up in item units).
 bool stream_plan(const Plan &p, GroupedArgs &A) {
     const long long sms = sm_count();
     long long best_cost = -1;
@@ -878,7 +958,7 @@ bool stream_plan(const Plan &p, GroupedArgs &A) {
         if (per_sm < kGOnePhaseMinBlocks) continue;
         const long long slots = (long long)per_sm * sms;
         const long long blocks = (long long)T.N * T.G * T.n_rb;
-        const long long cost = ceil_div(blocks, slots) * (T.JB + 2);
+        const long long cost = ceil_div(blocks, slots) * (ceil_div((long long)T.JB * T.n_seg32, kGWarps - 1) + 1);
         if (best_cost < 0 || cost < best_cost) {
             best_cost = cost;
             best_jb = jb;
