@@ -573,6 +573,23 @@ def test_dense_tc_pair_fp32_random_sweep():
     assert ran >= 15, ran
 
 
+@pytest.mark.parametrize("case", [
+    # 128-position tiles of two input rows (W = 64), padded origin (1, 1)
+    dict(x_shape=[2, 64, 8, 64], w_shape=[64, 32, 4, 4], strides=[2, 2], pads=[1, 1, 1, 1], bias=True),
+    # W = 32 (four rows per tile), 72 channels (a partial 64-channel block), stride 1
+    dict(x_shape=[1, 72, 4, 32], w_shape=[72, 16, 3, 3], strides=[1, 1], pads=[1, 1, 1, 1], bias=True),
+    # W = 128 (one row per tile), a 1x1 kernel: no halo, padded origin 0
+    dict(x_shape=[2, 128, 4, 128], w_shape=[128, 32, 1, 1], strides=[1, 1], bias=False),
+    # 3-D on the pair kernel, k = s (no halo), 16 x 16 slices
+    dict(x_shape=[1, 64, 2, 8, 16], w_shape=[64, 16, 2, 2, 2], strides=[2, 2, 2], bias=True),
+])
+def test_dense_tc_pair_whole_row_tiles(case):
+    """fp16 channels-first shapes whose 128-position re-layout tiles are whole
+    input rows (W of 32, 64 or 128), with and without a halo, a partial
+    64-channel block and a 3-D volume: the whole output against the oracle."""
+    full_parity(case, torch.float16, 91, "nchw", algo="dense_tc_pair", expect_kernel="dense_tc_pair")
+
+
 @pytest.mark.parametrize("dtype,case", [
     (torch.float16, dict(x_shape=[2, 64, 11, 13], w_shape=[64, 72, 4, 4], strides=[2, 2], pads=[1, 1, 1, 1],
                          bias=True)),
