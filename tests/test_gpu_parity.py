@@ -396,6 +396,20 @@ def test_grouped_one_phase_path(case):
     # output_padding on both axes
     dict(x_shape=[2, 32, 12, 16], w_shape=[32, 16, 1, 1], strides=[3, 2], pads=[0, 0, 0, 0],
          output_padding=[2, 1], group=2, bias=True),
+    # dilation 2 with kernels of 2 and 3 taps, 16 and 32 channels per group:
+    # 2, 4, 6, 8 and 12 (tap, 16-channel step) MMA steps per output tile
+    dict(x_shape=[2, 32, 12, 16], w_shape=[32, 16, 1, 2], strides=[2, 2], dilations=[2, 2], pads=[0, 0, 0, 1],
+         group=2, bias=True),
+    dict(x_shape=[2, 32, 12, 16], w_shape=[32, 16, 2, 2], strides=[2, 2], dilations=[2, 2], pads=[0, 0, 0, 1],
+         group=2, bias=True, activation="relu"),
+    dict(x_shape=[2, 32, 12, 16], w_shape=[32, 16, 2, 3], strides=[2, 2], dilations=[2, 2], pads=[0, 1, 0, 2],
+         group=2, bias=True),
+    dict(x_shape=[2, 64, 12, 16], w_shape=[64, 16, 2, 2], strides=[2, 2], dilations=[2, 2], pads=[0, 0, 0, 1],
+         group=2, bias=True),
+    dict(x_shape=[2, 64, 12, 16], w_shape=[64, 16, 2, 3], strides=[2, 2], dilations=[2, 2], pads=[0, 1, 0, 2],
+         group=2, bias=False),
+    # rank 1, four taps
+    dict(x_shape=[4, 96, 64], w_shape=[96, 16, 4], strides=[2], dilations=[2], pads=[0, 5], group=6, bias=True),
 ])
 def test_grouped_stream_path(case):
     """One-phase grouped shapes with 16-byte output rows (out_x % 8 == 0, at
