@@ -247,6 +247,31 @@ def test_kernel_selection(x_shape, w_shape, dtype, layout, kernel):
     assert wb > 0 and ws >= 0
 
 
+def test_kernel_selection_workloads_and_one_by_one():
+    """The kernel each workload is measured on (host planning only), and the
+    1x1 rule: 1x1 stride-1 fp16 channels-first shapes whose output rows are a
+    multiple of 8 wide plan to the halo kernel (row mode), other widths to the
+    pair kernel."""
+    want = {1: "generic", 2: "dense_tc_pair", 3: "dense_tc", 4: "dense_tc_pair", 5: "grouped"}
+    for wid, kernel in want.items():
+        wl = WORKLOADS[wid]
+        case = dict(x_shape=wl.x_shape, w_shape=wl.w_shape, strides=wl.strides,
+                    dilations=wl.dilations, pads=wl.pads, output_padding=wl.output_padding,
+                    auto_pad=wl.auto_pad, group=wl.group, bias=wl.bias)
+        plan = ct.ct_plan(_desc_from_case(case, dtype=wl.dtype))
+        try:
+            assert ct.ct_plan_kernel(plan) == kernel, (wid, ct.ct_plan_kernel(plan))
+        finally:
+            ct.ct_plan_destroy(plan)
+    k, _, _ = _kernel_for([8, 512, 64, 64], [512, 256, 1, 1], torch.float16, strides=[1, 1])
+    assert k == "dense_tc"
+    k, _, _ = _kernel_for([4, 128, 20, 20], [128, 64, 1, 1], torch.float16, strides=[1, 1])
+    assert k == "dense_tc_pair"
+    # a 1x1 kernel with stride 2 is not a plain GEMM: the pair kernel
+    k, _, _ = _kernel_for([8, 256, 32, 32], [256, 128, 1, 1], torch.float16, strides=[2, 2])
+    assert k == "dense_tc_pair"
+
+
 def test_pair_kernel_sizes():
     """Workspace and packed-weight sizes of the pair kernel: the padded
     channels-last copy (two planes for fp32) and one packed tile per
